@@ -1,0 +1,67 @@
+"""Seeded synthetic inputs shared by the tests, the bench and the oracle checks.
+
+This module holds no arithmetic of the attention method: it only draws Gaussian
+Q/K/V, optionally RMS-normalises Q and K per head vector (the stand-in for the
+Wan2.1 QK-RMSNorm that precedes attention in the target DiTs), and rounds to
+the storage dtype.  Both the CUDA path and the oracle consume its output.
+
+Recipe (one independent numpy PCG64 stream per tensor and head, so any head can
+be regenerated alone for sampled-row checks):
+  stream(seed, which, b, h) = default_rng(SeedSequence([seed, which, b, h]))
+  which: 0 = q, 1 = k, 2 = v;  x = scale * standard_normal((N, d)) in float64
+  rms_qk: q, k -> x / sqrt(mean(x**2, axis=-1) + 1e-6)
+  storage: float32, then bfloat16 by round-to-nearest-even (torch's cast).
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+WHICH = {"q": 0, "k": 1, "v": 2}
+
+
+def head_array(seed: int, which: str, b: int, h: int, N: int, d: int,
+               scale: float = 1.0, rms_qk: bool = False) -> np.ndarray:
+    """float64 [N, d] draw for one (tensor, batch, head)."""
+    rng = np.random.default_rng(np.random.SeedSequence([seed, WHICH[which], b, h]))
+    x = rng.standard_normal((N, d)) * scale
+    if rms_qk and which in ("q", "k"):
+        x = x / np.sqrt(np.mean(x * x, axis=-1, keepdims=True) + 1e-6)
+    return x
+
+
+def _store(x64: np.ndarray, dtype: str) -> torch.Tensor:
+    t = torch.from_numpy(x64.astype(np.float32))
+    if dtype == "bf16":
+        return t.to(torch.bfloat16)
+    if dtype == "f32":
+        return t
+    raise ValueError(dtype)
+
+
+def make_qkv(B: int, H: int, N: int, d: int, seed: int, dtype: str = "bf16",
+             scale: float = 1.0, rms_qk: bool = False, scales=None):
+    """Host tensors q, k, v of shape [B, H, N, d] in the storage dtype.
+
+    scales: optional (sq, sk, sv) overriding ``scale`` per tensor (used to
+    push the softmax branch to dominate, or the linear branch).
+    """
+    sc = scales if scales is not None else (scale, scale, scale)
+    out = []
+    for which, s in zip(("q", "k", "v"), sc):
+        t = torch.empty((B, H, N, d), dtype=torch.bfloat16 if dtype == "bf16" else torch.float32)
+        for b in range(B):
+            for h in range(H):
+                t[b, h] = _store(head_array(seed, which, b, h, N, d, s, rms_qk), dtype)
+        out.append(t)
+    return tuple(out)
+
+
+def make_state(B: int, H: int, d: int, seed: int, scale: float = 1.0):
+    """A non-negative z and arbitrary S, fp32, shaped like a recurrent state
+    ([B,H,2d,d], [B,H,2d]); used only to exercise the step call from a
+    non-zero starting state."""
+    rng = np.random.default_rng(np.random.SeedSequence([seed, 7]))
+    S = rng.standard_normal((B, H, 2 * d, d)) * scale
+    z = np.abs(rng.standard_normal((B, H, 2 * d))) * scale + 1.0
+    return torch.from_numpy(S.astype(np.float32)), torch.from_numpy(z.astype(np.float32))
