@@ -1,0 +1,453 @@
+#!/usr/bin/env python
+"""Benchmark of ReHyAt's temporally chunked hybrid attention forward on B200.
+
+Default workload (one GPU): Wan2.1-1.3B 480p attention shape, B=1, H=12,
+d=128, F=21 latent frames x 30x52 = 1560 tokens (32,760 tokens), T_c=3,
+T_o=1, bf16, Gaussian Q/K/V with RMS-normalised Q/K (seeded, synthetic).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--config wan13b|wan14b|recurrent] [--sweep]
+
+A step = one pass of the whole path over one batch: the states stage
+(phi(K), per-segment phi(K)^T V, chunk scan) and the fused chunk attention.
+Under torchrun each rank runs its own batch (weak scaling, no collective on
+the data path); the step time is the max over ranks.  Rank 0 prints one JSON
+line.  --impl reference times the fp64 CPU oracle on bounded row samples.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "hybrid-attention tokens/s on 1 B200 and % of roofline, Wan2.1-1.3B 480p shape"
+UNIT = "tokens/s"
+
+CONFIGS = {
+    "wan13b": dict(workload="Wan2.1-1.3B 480p attention shape", B=1, H=12, d=128, F=21, S_tok=1560,
+                   T_c=3, T_o=1, seed=1),
+    "wan14b": dict(workload="Wan2.1-14B 720p-like attention shape", B=1, H=40, d=128, F=21, S_tok=3600,
+                   T_c=3, T_o=1, seed=3),
+    "recurrent": dict(workload="long-video recurrent mode (rehyat_step), 81 latent frames", B=1, H=12, d=128,
+                      F=81, S_tok=1560, T_c=3, T_o=1, seed=2),
+}
+SWEEP = [(F, tc, to) for (tc, to) in ((2, 1), (3, 1), (5, 2)) for F in (21, 41, 81, 161)]
+
+
+# --------------------------------------------------------------------------- #
+# algorithmic work (FLOPs and bytes the method needs, nothing masked counted)  #
+# --------------------------------------------------------------------------- #
+def chunks(F, S, Tc, To):
+    tc, to = min(Tc, F), min(To, F)
+    N, Np = F * S, tc * S
+    for t in range(-(-F // tc)):
+        q0, q1 = t * Np, min((t + 1) * Np, N)
+        yield q0, q1, max(q0 - to * S, 0), q1
+
+
+def work(c):
+    B, H, d, F, S, Tc, To = (c[k] for k in ("B", "H", "d", "F", "S_tok", "T_c", "T_o"))
+    BH, N, D2 = B * H, F * S, 2 * d
+    ch = list(chunks(F, S, Tc, To))
+    pairs = sum((q1 - q0) * (hi - lo) for q0, q1, lo, hi in ch)
+    n_lin = sum(q1 - q0 for q0, q1, lo, hi in ch if lo > 0)       # queries with a linear term
+    folded = max(lo for _, _, lo, _ in ch)                        # keys folded into states
+    attn_flops = BH * (4 * d * pairs + 2 * D2 * (d + 1) * n_lin)
+    state_flops = BH * 2 * D2 * (d + 1) * folded
+    attn_bytes = BH * N * d * 2 * 4 + BH * len(ch) * D2 * (d * 4 + 4)     # q,k,v,out + states (hi,lo,z)
+    state_bytes = BH * folded * d * 2 * 2 + BH * len(ch) * D2 * (d * 4 + 4)
+    return dict(pairs_per_head=pairs, attn_flops=attn_flops, state_flops=state_flops, attn_bytes=attn_bytes,
+                state_bytes=state_bytes, tokens=B * N)
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as fh:
+            j = json.load(fh)
+        return j["bf16_tflops"], j.get("bf16_tflops_sustained"), j["hbm_gbs"], "measured"
+    except Exception:
+        return 1590.0, 1400.0, 6650.0, "fallback"
+
+
+# --------------------------------------------------------------------------- #
+# clocks sampled during the timed region (NVML reads only)                    #
+# --------------------------------------------------------------------------- #
+class ClockSampler:
+    REASONS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown",
+               0x4: "sw_power_cap", 0x80: "hw_power_brake_slowdown", 0x1: "gpu_idle"}
+
+    def __init__(self, index):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self.nv = None
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                r = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for bit, name in self.REASONS.items():
+                    if r & bit and name != "gpu_idle":
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(0.005)
+
+    def __enter__(self):
+        if self.nv is not None:
+            self.th = threading.Thread(target=self._run, daemon=True)
+            self.th.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self.nv is not None:
+            self.th.join()
+
+    def summary(self):
+        med = statistics.median(self.samples) if self.samples else None
+        return {"sm_mhz": med, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                "samples": len(self.samples)}
+
+
+# --------------------------------------------------------------------------- #
+# CPU baseline: the fp64 oracle on bounded row samples                         #
+# --------------------------------------------------------------------------- #
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return len(os.sched_getaffinity(0))
+
+
+def oracle_sample_rate(c, q, k, v, budget_s):
+    """Tokens/s of the oracle: rows (all heads) per second on a row sample
+    sized to take about budget_s seconds.  Returns (rate, rows, seconds)."""
+    import numpy as np
+    import oracle.rehyat_oracle as orc
+    N = c["F"] * c["S_tok"]
+    rng = np.random.default_rng(7)
+    args = (c["F"], c["S_tok"], c["T_c"], c["T_o"])
+    t0 = time.perf_counter()
+    orc.oracle_forward(q, k, v, *args, rows=np.sort(rng.choice(N, 8, replace=False)))
+    t8 = time.perf_counter() - t0
+    n = int(max(8, min(N, 8 * budget_s / max(t8, 1e-3))))
+    rows = np.sort(rng.choice(N, n, replace=False))
+    t0 = time.perf_counter()
+    orc.oracle_forward(q, k, v, *args, rows=rows)
+    dt = time.perf_counter() - t0
+    return n / dt, n, dt
+
+
+# --------------------------------------------------------------------------- #
+# our arm                                                                      #
+# --------------------------------------------------------------------------- #
+def dist_env():
+    return int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)), int(os.environ.get("LOCAL_RANK", 0))
+
+
+def max_over_ranks(x, world, dev):
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def run_forward_bench(args, c, rank, world, dev):
+    import torch
+    from linear_attention_video_chunk_b200 import inputs
+    from linear_attention_video_chunk_b200 import rehyat as R
+    B, H, d, F, S, Tc, To = (c[k] for k in ("B", "H", "d", "F", "S_tok", "T_c", "T_o"))
+    N = F * S
+    q, k, v = inputs.make_qkv(B, H, N, d, c["seed"] + 1000 * rank, rms_qk=True, pin=True)
+    qd, kd, vd = (x.to(dev, non_blocking=True) for x in (q, k, v))
+    out = torch.empty_like(qd)
+    ws = R.alloc_workspace(R.workspace_bytes(B, H, F, S, d, Tc, To), dev)
+    torch.cuda.synchronize()
+
+    def step(e0=None, e1=None, e2=None):
+        if e0 is not None:
+            e0.record()
+        R.forward_states(kd, vd, F, S, Tc, To, ws)
+        if e1 is not None:
+            e1.record()
+        R.forward_attention(qd, kd, vd, F, S, Tc, To, out, ws)
+        if e2 is not None:
+            e2.record()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(dev.index if dev.index is not None else 0) as clk:
+        start.record()
+        for i in range(K):
+            step(*ev[i])
+        end.record()
+        torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    ms_step = max_over_ranks(start.elapsed_time(end) / K, world, dev)
+    attn_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in ev)
+    state_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
+
+    # end to end through the public API: pinned host inputs -> device ->
+    # forward -> result back to pinned host memory, every step
+    out_h = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+    Ke = max(3, min(K, 20))
+    for _ in range(2):
+        for src, dst in ((q, qd), (k, kd), (v, vd)):
+            dst.copy_(src, non_blocking=True)
+        R.forward(qd, kd, vd, F, S, Tc, To, out=out, workspace=ws)
+        out_h.copy_(out, non_blocking=True)
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s2.record()
+    for _ in range(Ke):
+        for src, dst in ((q, qd), (k, kd), (v, vd)):
+            dst.copy_(src, non_blocking=True)
+        R.forward(qd, kd, vd, F, S, Tc, To, out=out, workspace=ws)
+        out_h.copy_(out, non_blocking=True)
+    e2.record()
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(s2.elapsed_time(e2) / Ke, world, dev)
+    status = R.device_status()
+    if status != R.OK:
+        raise RuntimeError(f"device status {R.status_string(status)}")
+    return dict(ms_step=ms_step, attn_ms=attn_ms, state_ms=state_ms, e2e_ms=e2e_ms, clocks=clk.summary(),
+                h2d=3 * q.numel() * q.element_size(), d2h=out.numel() * out.element_size(), q=q, k=k, v=v,
+                launches=3 * K)
+
+
+def run_ours(args):
+    import torch
+    rank, world, local = dist_env()
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    c = dict(CONFIGS[args.config])
+    if args.config == "recurrent":
+        res = run_recurrent_bench(args, c, rank, world, dev)
+    else:
+        res = run_forward_bench(args, c, rank, world, dev)
+    w = work(c)
+    bf16_peak, bf16_sus, hbm, src = peaks()
+    tokens = w["tokens"] * world
+    line = {
+        "metric": METRIC, "value": tokens / (res["ms_step"] / 1e3), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": res["ms_step"], "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic: seeded N(0,1) Q/K/V, per-vector RMS-normalised Q/K, bf16 (no latents or weights)",
+        "config": {"workload": c["workload"], "B": c["B"], "H": c["H"], "d": c["d"], "F": c["F"],
+                   "S_tok": c["S_tok"], "chunk_frames": c["T_c"], "overlap_frames": c["T_o"],
+                   "tokens_per_step_per_gpu": w["tokens"], "parallelism": f"replicas x{world} (no collective)",
+                   "l2": "inputs larger than L2: q+k+v = %.0f MB per GPU" % (3 * w["tokens"] * c["H"] * c["d"] * 2 / 1e6)},
+    }
+    if args.config != "recurrent":
+        achieved = w["attn_flops"] / (res["attn_ms"] / 1e3) / 1e12
+        line["roofline"] = {
+            "kernel": "hybrid_chunk_attn_kernel", "bound": "tensor", "achieved": achieved, "peak": bf16_peak,
+            "unit": "TFLOP/s", "frac": achieved / bf16_peak, "peak_source": f"{src} bf16 dense (burst)",
+            "frac_of_sustained": achieved / bf16_sus if bf16_sus else None, "traffic": None,
+            "kernel_ms": res["attn_ms"], "flops_per_launch": w["attn_flops"],
+            "states_stage_ms": res["state_ms"],
+            "path_frac": (w["attn_flops"] + w["state_flops"]) / (res["ms_step"] / 1e3) / 1e12 / bf16_peak,
+        }
+    line["e2e"] = {"value": tokens / (res["e2e_ms"] / 1e3), "unit": UNIT, "h2d_bytes_per_step": res["h2d"],
+                   "d2h_bytes_per_step": res["d2h"], "ms_per_step": res["e2e_ms"]}
+    line["clocks"] = res["clocks"]
+    line["gpu_launches"] = res["launches"]
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and args.config == "wan13b":
+        rate, n, dt = oracle_sample_rate(c, res["q"], res["k"], res["v"], args.cpu_budget)
+        line["cpu_baseline"] = {"value": rate, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+                                "sample": f"fp64 explicit-mask oracle on {n} random query rows x all {c['H']} "
+                                          f"heads of the same workload ({dt:.1f} s); value = rows/s"}
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def run_recurrent_bench(args, c, rank, world, dev):
+    """F frames streamed chunk by chunk through rehyat_step; device memory
+    must stay flat across steps (state is constant-size)."""
+    import torch
+    from linear_attention_video_chunk_b200 import inputs
+    from linear_attention_video_chunk_b200 import rehyat as R
+    B, H, d, F, S, Tc, To = (c[k] for k in ("B", "H", "d", "F", "S_tok", "T_c", "T_o"))
+    q, k, v = inputs.make_qkv(B, H, F * S, d, c["seed"] + 1000 * rank, rms_qk=True, pin=True)
+    qd, kd, vd = (x.to(dev) for x in (q, k, v))
+    nc = -(-F // Tc)
+    slices = []
+    for t in range(nc):
+        f0, w0, cf, qf, ef = R.step_frames(t, F, Tc, To)
+        slices.append((qd[:, :, f0 * S:(f0 + qf) * S].contiguous(), kd[:, :, w0 * S:(f0 + qf) * S].contiguous(),
+                       vd[:, :, w0 * S:(f0 + qf) * S].contiguous(), qf, cf, ef))
+    Sst = torch.zeros(B, H, 2 * d, d, device=dev)
+    zst = torch.zeros(B, H, 2 * d, device=dev)
+    ws = R.alloc_workspace(max(R.step_workspace_bytes(B, H, S, d, s[3], s[4], s[5]) for s in slices), dev)
+    outs = [torch.empty_like(s[0]) for s in slices]
+
+    def video():
+        Sst.zero_()
+        zst.zero_()
+        for (qc, kc, vc, qf, cf, ef), o in zip(slices, outs):
+            R.step(qc, kc, vc, Sst, zst, S, qf, cf, ef, out=o, workspace=ws)
+
+    for _ in range(max(1, args.warmup // 3)):
+        video()
+    torch.cuda.synchronize()
+    K = max(1, args.steps // 10)
+    s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(dev.index or 0) as clk:
+        s0.record()
+        for _ in range(K):
+            video()
+        s1.record()
+        torch.cuda.synchronize()
+    ms = max_over_ranks(s0.elapsed_time(s1) / K, world, dev)
+    return dict(ms_step=ms, e2e_ms=ms, clocks=clk.summary(), h2d=0, d2h=0, launches=K * nc * 4, q=q, k=k, v=v)
+
+
+def run_sweep(args):
+    import numpy as np
+    import torch
+    from linear_attention_video_chunk_b200 import inputs
+    from linear_attention_video_chunk_b200 import rehyat as R
+    dev = torch.device("cuda", 0)
+    bf16_peak, _, _, src = peaks()
+    B, H, d, S = 2, 12, 128, 1560
+    res = {}
+    for F, Tc, To in SWEEP:
+        q, k, v = (x.to(dev) for x in inputs.make_qkv(B, H, F * S, d, 100 + len(res), rms_qk=True))
+        out = torch.empty_like(q)
+        ws = R.alloc_workspace(R.workspace_bytes(B, H, F, S, d, Tc, To), dev)
+        for _ in range(3):
+            R.forward(q, k, v, F, S, Tc, To, out=out, workspace=ws)
+        torch.cuda.synchronize()
+        K = 10
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(K):
+            R.forward(q, k, v, F, S, Tc, To, out=out, workspace=ws)
+        e1.record()
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / K
+        w = work(dict(B=B, H=H, d=d, F=F, S_tok=S, T_c=Tc, T_o=To))
+        frac = (w["attn_flops"] + w["state_flops"]) / (ms / 1e3) / 1e12 / bf16_peak
+        res[(F, Tc, To)] = ms
+        print(json.dumps({"sweep_point": {"B": B, "H": H, "F": F, "T_c": Tc, "T_o": To}, "ms": ms,
+                          "tokens_per_s": B * F * S / (ms / 1e3), "roofline_frac": frac,
+                          "peak": f"{bf16_peak} TFLOP/s {src}"}), flush=True)
+        del q, k, v, out, ws
+        torch.cuda.empty_cache()
+    for Tc, To in ((2, 1), (3, 1), (5, 2)):
+        Fs = np.array([F for F, a, b in SWEEP if (a, b) == (Tc, To)], dtype=float)
+        ts = np.array([res[(F, Tc, To)] for F in Fs.astype(int)])
+        A = np.stack([Fs, np.ones_like(Fs)], 1)
+        coef, *_ = np.linalg.lstsq(A, ts, rcond=None)
+        r2 = 1 - ((A @ coef - ts) ** 2).sum() / ((ts - ts.mean()) ** 2).sum()
+        print(json.dumps({"linear_fit": {"T_c": Tc, "T_o": To, "ms_per_frame": coef[0], "intercept_ms": coef[1],
+                                         "r2": r2}}), flush=True)
+
+
+# --------------------------------------------------------------------------- #
+# reference arm: the fp64 oracle on the host cores                             #
+# --------------------------------------------------------------------------- #
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return
+    from linear_attention_video_chunk_b200 import inputs
+    c = dict(CONFIGS["wan13b"])
+    B, H, d, F, S = (c[k] for k in ("B", "H", "d", "F", "S_tok"))
+    q, k, v = inputs.make_qkv(B, H, F * S, d, c["seed"], rms_qk=True)
+    import numpy as np
+    import oracle.rehyat_oracle as orc
+    N = F * S
+    rng = np.random.default_rng(11)
+    per_step_budget = max(0.2, 150.0 / max(1, args.steps + args.warmup))
+    # size each step's row sample from a calibration call
+    t0 = time.perf_counter()
+    orc.oracle_forward(q, k, v, F, S, c["T_c"], c["T_o"], rows=np.arange(4))
+    t4 = time.perf_counter() - t0
+    n = int(max(1, min(N, 4 * per_step_budget / max(t4, 1e-3))))
+    times = []
+    for i in range(args.warmup + args.steps):
+        rows = np.sort(rng.choice(N, n, replace=False))
+        t0 = time.perf_counter()
+        orc.oracle_forward(q, k, v, F, S, c["T_c"], c["T_o"], rows=rows)
+        if i >= args.warmup:
+            times.append(time.perf_counter() - t0)
+    sec = sum(times) / len(times)
+    val = n / sec
+    line = {
+        "impl": "reference", "metric": METRIC, "value": val, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": sec * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic (same generator and seed as the GPU arm)",
+        "config": {"workload": c["workload"], "B": B, "H": H, "d": d, "F": F, "S_tok": S,
+                   "chunk_frames": c["T_c"], "overlap_frames": c["T_o"]},
+        "cpu_baseline": {"value": val, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+                         "sample": f"each step: fp64 explicit-mask oracle on {n} random query rows x all {H} heads"},
+        "e2e": {"value": val, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--config", choices=tuple(CONFIGS), default="wan13b")
+    ap.add_argument("--sweep", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work for cpu_baseline")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+    elif args.sweep:
+        run_sweep(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

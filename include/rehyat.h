@@ -1,0 +1,202 @@
+/*
+ * rehyat.h -- C ABI of the B200 (sm_100a) implementation of ReHyAt's
+ * temporally chunked hybrid attention forward.
+ *
+ * Source of every operation: "ReHyAt: Recurrent Hybrid Attention for Video
+ * Diffusion Transformers" (Ghafoorian & Habibian, arXiv 2601.04342):
+ *   §3.1  linear attention y_i = phi(q_i) sum_j phi(k_j) v_j^T / phi(q_i) sum_j phi(k_j),
+ *         the two sums cached independently of i; phi non-negative, 1 + elu.
+ *   §3.2  hybrid output y = (a^S + a^L) / (n^S + n^L) (joint normaliser);
+ *         chunk sets T^S_t, T^L_t with and without overlap;
+ *         polynomial feature map phi(x) = [psi_1(x)^1, ..., psi_P(x)^P].
+ *   §3.3  Recurrent HyAt: T^L_t = { j < max(tN' - T_o HW, 0) },
+ *         T^S_t = { max(tN' - T_o HW, 0) <= j < (t+1)N' }.
+ *
+ * Readings taken where the text is silent (the paper's prose around the
+ * equations is lost):
+ *   - N' = chunk_frames * S_tok; chunk t owns queries [tN', min((t+1)N', N)).
+ *   - tokens are frame-major: j = f * S_tok + spatial index; N = F * S_tok.
+ *   - the last chunk is ragged when F is not a multiple of chunk_frames.
+ *   - phi(x) = [psi(x), psi(x)^2] with psi = 1 + elu on both q and k (P = 2,
+ *     D' = 2d): the only concrete psi the paper gives.
+ *   - softmax weight exp(q.k / sqrt(d)).
+ *   - every call computes the §3.3 (causal / recurrent) sets, so the parallel
+ *     form and the step form compute the same function.
+ *
+ * Conventions for every entry point:
+ *   - Tensors are dense, row-major, in DEVICE memory owned by the caller:
+ *     q, k, v, out are [B, H, N, d] (d fastest).  bf16 entry points take
+ *     `const void*` pointing at IEEE bfloat16 data; _f32 ones take float.
+ *     All device pointers must be 16-byte aligned (TMA requirement).
+ *   - d must be 64 or 128 (REHYAT_EUNSUPPORTED otherwise).
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Calls are asynchronous: they validate, launch and return;
+ *     outputs are valid once the stream reaches that point.  No host sync.
+ *   - Validation failures return a status and launch nothing.  Launch
+ *     failures return REHYAT_ECUDA.  Entry points without a `workspace`
+ *     argument allocate stream-ordered scratch (cudaMallocAsync /
+ *     cudaFreeAsync on `stream`); the _ws variants allocate nothing.
+ *   - Device-side waits are bounded (about 2 s).  A wait that runs out sets
+ *     a device error word, the kernel returns early (its outputs are then
+ *     invalid), and rehyat_device_status() reports REHYAT_ETIMEOUT.
+ *   - Results are deterministic: no atomics on the data path.
+ *   - Multiple calls may run concurrently on different streams.
+ */
+#ifndef REHYAT_H
+#define REHYAT_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  REHYAT_OK = 0,
+  REHYAT_EINVAL = 1,        /* bad argument: null/misaligned pointer, size < 1, overflow */
+  REHYAT_EUNSUPPORTED = 2,  /* valid but not implemented here (d not in {64,128}) */
+  REHYAT_ENOMEM = 3,        /* workspace allocation failed / workspace too small */
+  REHYAT_ECUDA = 4,         /* a CUDA runtime/driver call or launch failed */
+  REHYAT_ETIMEOUT = 5       /* a bounded device-side wait ran out (see rehyat_device_status) */
+} rehyat_status;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* rehyat_status_string(int status);
+
+/* ---------------------------------------------------------------------- *
+ * Parallel form (§3.2 joint normaliser over the §3.3 sets), whole video.  *
+ * ---------------------------------------------------------------------- */
+
+/* bf16 forward on tensor cores (tcgen05/TMEM, TMA).
+ * q, k, v: [B,H,N,d] bf16 with N = F*S_tok.  out: [B,H,N,d] bf16.
+ * chunk_frames = T_c >= 1, overlap_frames = T_o >= 0 (any value, also >= T_c).
+ * Arithmetic: bf16 operands, fp32 accumulation, fp32 softmax and combine;
+ * the linear state is kept in fp32 and fed to the tensor cores as a bf16
+ * hi + lo pair. */
+int rehyat_forward(const void* q, const void* k, const void* v,
+                   int B, int H, int F, int S_tok, int d,
+                   int chunk_frames, int overlap_frames,
+                   void* out, void* stream);
+
+/* Bytes of scratch rehyat_forward_ws needs for this shape. */
+int rehyat_forward_workspace_bytes(int B, int H, int F, int S_tok, int d,
+                                   int chunk_frames, int overlap_frames,
+                                   size_t* bytes);
+
+/* rehyat_forward with caller-provided device scratch (>= the size above,
+ * 256-byte aligned); allocates nothing.  The workspace is overwritten. */
+int rehyat_forward_ws(const void* q, const void* k, const void* v,
+                      int B, int H, int F, int S_tok, int d,
+                      int chunk_frames, int overlap_frames,
+                      void* out, void* workspace, size_t workspace_bytes,
+                      void* stream);
+
+/* The two stages of rehyat_forward_ws, callable separately (same kernels):
+ *   states:    phi(K), per-segment phi(K)^T V and sum phi(K), exclusive scan
+ *              over chunks -> the state S_t, z_t entering each chunk, written
+ *              into the workspace;
+ *   attention: the fused per-chunk kernel (local softmax + phi(Q) S_t,
+ *              phi(Q) z_t, joint normaliser), reading the states from the
+ *              workspace filled by the states stage for the same shape. */
+int rehyat_forward_states(const void* k, const void* v,
+                          int B, int H, int F, int S_tok, int d,
+                          int chunk_frames, int overlap_frames,
+                          void* workspace, size_t workspace_bytes, void* stream);
+int rehyat_forward_attention(const void* q, const void* k, const void* v,
+                             int B, int H, int F, int S_tok, int d,
+                             int chunk_frames, int overlap_frames,
+                             void* out, void* workspace, size_t workspace_bytes,
+                             void* stream);
+
+/* fp32 forward (SIMT fp32 throughout, accurate exp); same sets and layout.
+ * Meant for small problems and tight-tolerance checks; any size is legal. */
+int rehyat_forward_f32(const float* q, const float* k, const float* v,
+                       int B, int H, int F, int S_tok, int d,
+                       int chunk_frames, int overlap_frames,
+                       float* out, void* stream);
+
+/* Diagnostic form of rehyat_forward: runs the same fused tensor-core kernel
+ * but writes the unnormalised terms of the §3.2 joint normaliser instead of
+ * their ratio, all fp32, scaled by exp(-M):
+ *   aS [B,H,N,d] = sum_{T^S} exp(s - M) v      nS [B,H,N] = sum_{T^S} exp(s - M)
+ *   aL [B,H,N,d] = exp(-M) phi(q) S_t          nL [B,H,N] = exp(-M) phi(q) z_t
+ *   M  [B,H,N]   = the shift used (natural log units), s = q.k/sqrt(d).
+ * y = (aS + aL) / (nS + nL).  aL (and nL) are 0 where T^L_t is empty. */
+int rehyat_forward_parts(const void* q, const void* k, const void* v,
+                         int B, int H, int F, int S_tok, int d,
+                         int chunk_frames, int overlap_frames,
+                         float* aS, float* nS, float* aL, float* nL, float* M,
+                         void* stream);
+
+/* States entering each chunk, exported for inspection (bf16 inputs,
+ * tensor-core phi(K)^T V, fp32 scan):  S [B,H,n_chunks,2d,d] fp32,
+ * z [B,H,n_chunks,2d] fp32 with n_chunks = ceil(F / chunk_frames);
+ * S_t = sum_{j < lo_t} phi(k_j) v_j^T, z_t = sum_{j < lo_t} phi(k_j). */
+int rehyat_chunk_states(const void* k, const void* v,
+                        int B, int H, int F, int S_tok, int d,
+                        int chunk_frames, int overlap_frames,
+                        float* S, float* z, void* stream);
+
+/* ---------------------------------------------------------------------- *
+ * Recurrent form (§3.3 chunk-wise RNN), one chunk per call.               *
+ * ---------------------------------------------------------------------- */
+
+/* One chunk of the recurrent form with a constant-size state.
+ *   q_c: [B,H,q_frames*S_tok,d]   the chunk's queries.
+ *   k_c, v_c: [B,H,(ctx_frames+q_frames)*S_tok,d]  its whole softmax window:
+ *        ctx_frames overlap frames followed by the chunk's own frames.
+ *   state_S: [B,H,2d,d] fp32, state_z: [B,H,2d] fp32: the linear state of
+ *        every key before the window (caller-owned; zero before chunk 0),
+ *        updated IN PLACE: after the attention, the first evict_frames frames
+ *        of k_c/v_c are folded in (S += phi(K)^T V, z += sum phi(K)).
+ *   out_c: [B,H,q_frames*S_tok,d].
+ * For chunk t of a video with window start w_t = max(t*T_c - T_o, 0):
+ *   ctx_frames = t*T_c - w_t, q_frames = min(T_c, F - t*T_c),
+ *   evict_frames = w_{t+1} - w_t   (w_{t+1} clipped to the window end).
+ * 0 <= evict_frames <= ctx_frames + q_frames.  bf16 in, fp32 state. */
+int rehyat_step(const void* q_c, const void* k_c, const void* v_c,
+                float* state_S, float* state_z, void* out_c,
+                int B, int H, int S_tok, int d,
+                int q_frames, int ctx_frames, int evict_frames, void* stream);
+
+int rehyat_step_workspace_bytes(int B, int H, int S_tok, int d,
+                                int q_frames, int ctx_frames, int evict_frames,
+                                size_t* bytes);
+
+/* rehyat_step with caller-provided scratch; allocates nothing. */
+int rehyat_step_ws(const void* q_c, const void* k_c, const void* v_c,
+                   float* state_S, float* state_z, void* out_c,
+                   int B, int H, int S_tok, int d,
+                   int q_frames, int ctx_frames, int evict_frames,
+                   void* workspace, size_t workspace_bytes, void* stream);
+
+/* fp32 step (SIMT), same contract with float tensors. */
+int rehyat_step_f32(const float* q_c, const float* k_c, const float* v_c,
+                    float* state_S, float* state_z, float* out_c,
+                    int B, int H, int S_tok, int d,
+                    int q_frames, int ctx_frames, int evict_frames, void* stream);
+
+/* ---------------------------------------------------------------------- *
+ * Feature map and device status.                                          *
+ * ---------------------------------------------------------------------- */
+
+#define REHYAT_DTYPE_BF16 0
+#define REHYAT_DTYPE_F32 1
+
+/* §3.2 feature map phi(x) = [psi(x), psi(x)^2], psi = 1 + elu (§3.1),
+ * row-wise: x [rows, d] -> y [rows, 2d].  dtype codes REHYAT_DTYPE_*. */
+int rehyat_phi(const void* x, int x_dtype, void* y, int y_dtype,
+               int64_t rows, int d, void* stream);
+
+/* Synchronises the current device and reports whether any kernel of this
+ * library recorded a device-side error since the last call (REHYAT_ETIMEOUT
+ * when a bounded wait ran out), then clears the record.  *detail (optional)
+ * receives the raw error word (0 when clean). */
+int rehyat_device_status(unsigned int* detail);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* REHYAT_H */

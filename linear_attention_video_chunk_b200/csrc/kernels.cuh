@@ -1,0 +1,92 @@
+// kernels.cuh -- kernel parameter blocks and launchers (internal to librehyat).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "geom.cuh"
+
+namespace rehyat {
+
+// Fused per-chunk hybrid attention (tensor cores).  One CTA = one "unit":
+// up to two 128-row query tiles of one chunk of one (b,h).
+struct AttnParams {
+  CUtensorMap tm_q;   // [BH, N_q, D] bf16, box {64, 128, 1}, 128B swizzle
+  CUtensorMap tm_k;   // [BH, N_k, D]
+  CUtensorMap tm_v;   // [BH, N_k, D]
+  CUtensorMap tm_hi;  // [BH * state_mul, 2D, D] bf16: high part of S_t
+  CUtensorMap tm_lo;  // same: S_t - hi (rounded to bf16)
+  ChunkGeom g;
+  int BH;
+  int pairs;          // units per (bh, chunk)
+  int state_mul;      // state tile z-coordinate = bh * state_mul + (g.step ? 0 : t)
+  float scale_log2;   // log2(e) / sqrt(D)
+  const float* z;     // z_t (fp32); entry e of (bh, t) at z[bh*z_bh + t*z_t + e]
+  long long z_bh, z_t;
+  __nv_bfloat16* out; // [BH, N_q, D]
+  float* aS;          // diagnostic parts (PARTS kernels only)
+  float* nS;
+  float* aL;
+  float* nL;
+  float* Mo;
+};
+
+// phi(K)^T V and sum phi(K) over key segments (tensor cores).  One CTA =
+// one piece of one segment of one (b,h).
+struct StateParams {
+  CUtensorMap tm_k;   // [BH, N_k, D] bf16, box {64, 64, 1}
+  CUtensorMap tm_v;
+  SegGeom sg;
+  int BH;
+  float* part_S;      // [BH, n_seg, nsplit, 2D, D] fp32
+  float* part_z;      // [BH, n_seg, nsplit, 2D] fp32
+};
+
+// fp32 SIMT paths
+struct AttnF32Params {
+  ChunkGeom g;
+  int BH, D;
+  const float* q;     // [BH, N_q, D]
+  const float* k;     // [BH, N_k, D]
+  const float* v;
+  const float* S;     // S_t at S[bh*S_bh + t*S_t] ([2D, D] row-major)
+  long long S_bh, S_t;
+  const float* z;     // z_t at z[bh*z_bh + t*z_t]
+  long long z_bh, z_t;
+  float* out;         // [BH, N_q, D]
+};
+
+struct StateF32Params {
+  SegGeom sg;         // nsplit must be 1
+  int BH, D;
+  const float* k;
+  const float* v;
+  float* part_S;      // [BH, n_seg, 1, 2D, D]
+  float* part_z;
+};
+
+// Shared-memory bytes each tensor-core kernel needs (dynamic).
+int attn_smem_bytes(int D);
+int state_smem_bytes(int D);
+
+cudaError_t launch_attention(int D, bool parts, const AttnParams& p, int n_units, cudaStream_t s);
+cudaError_t launch_chunk_state(int D, const StateParams& p, int n_ctas, cudaStream_t s);
+// Exclusive prefix over segments (and sum over pieces): writes the state
+// entering each chunk, either as bf16 hi/lo (hi, lo non-null) or fp32 (Sf).
+cudaError_t launch_state_scan(const float* part_S, const float* part_z, int BH, int n_seg,
+                              int nsplit, int n_chunks, int D, __nv_bfloat16* hi,
+                              __nv_bfloat16* lo, float* Sf, float* zt, cudaStream_t s);
+// state_S/z += sum over pieces of one segment's partials.
+cudaError_t launch_state_accumulate(const float* part_S, const float* part_z, int BH, int nsplit,
+                                    int D, float* state_S, float* state_z, cudaStream_t s);
+// fp32 state -> bf16 hi/lo pair.
+cudaError_t launch_state_split(const float* S, long long n, __nv_bfloat16* hi, __nv_bfloat16* lo,
+                               cudaStream_t s);
+
+cudaError_t launch_attention_f32(const AttnF32Params& p, int n_chunks, cudaStream_t s);
+cudaError_t launch_chunk_state_f32(const StateF32Params& p, cudaStream_t s);
+cudaError_t launch_phi(const void* x, int x_f32, void* y, int y_f32, long long rows, int d,
+                       cudaStream_t s);
+
+}  // namespace rehyat

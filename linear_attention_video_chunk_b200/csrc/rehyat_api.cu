@@ -1,0 +1,536 @@
+// rehyat_api.cu -- the C ABI declared in include/rehyat.h: argument
+// validation, scratch planning, TMA tensor maps and kernel launches.  No
+// arithmetic of the method lives here.
+#include <climits>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "geom.cuh"
+#include "kernels.cuh"
+#include "rehyat.h"
+
+#define REHYAT_API extern "C" __attribute__((visibility("default")))
+
+namespace rehyat {
+cudaError_t read_and_clear_device_error(unsigned int* v);
+}
+
+namespace {
+using namespace rehyat;
+
+constexpr int kSplitTarget = 296;  // CTAs aimed at for the state kernels (2 waves of 148 SMs)
+
+// ---------------------------------------------------------------------------
+// validation
+// ---------------------------------------------------------------------------
+int check_ptr(const void* p) {
+  if (p == nullptr) return REHYAT_EINVAL;
+  if (reinterpret_cast<uintptr_t>(p) % 16 != 0) return REHYAT_EINVAL;
+  return REHYAT_OK;
+}
+
+int check_d(int d) {
+  if (d < 1) return REHYAT_EINVAL;
+  if (d != 64 && d != 128) return REHYAT_EUNSUPPORTED;
+  return REHYAT_OK;
+}
+
+// ---------------------------------------------------------------------------
+// plans
+// ---------------------------------------------------------------------------
+size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+struct FwdPlan {
+  int BH, N, D, nc, n_seg, nsplit, chunk_tok, ovl_tok, pairs, n_units;
+  size_t off_pS, off_pz, off_hi, off_lo, off_zt, bytes;       // bf16 path
+  size_t f32_off_pS, f32_off_pz, f32_off_S, f32_off_zt, f32_bytes;  // fp32 path
+};
+
+int plan_forward(int B, int H, int F, int S_tok, int d, int Tc, int To, FwdPlan* p) {
+  if (B < 1 || H < 1 || F < 1 || S_tok < 1 || Tc < 1 || To < 0) return REHYAT_EINVAL;
+  int st = check_d(d);
+  if (st != REHYAT_OK) return st;
+  const long long BH = static_cast<long long>(B) * H;
+  const long long N = static_cast<long long>(F) * S_tok;
+  if (BH > INT_MAX || N > INT_MAX / 2) return REHYAT_EINVAL;
+  if (BH * N * d > (1LL << 46)) return REHYAT_EINVAL;
+  // A chunk (or an overlap) longer than the video is the whole video.
+  const int tc = Tc < F ? Tc : F;
+  const int to = To < F ? To : F;
+  p->BH = static_cast<int>(BH);
+  p->N = static_cast<int>(N);
+  p->D = d;
+  p->chunk_tok = tc * S_tok;
+  p->ovl_tok = to * S_tok;
+  p->nc = cdiv(F, tc);
+  p->n_seg = p->nc - 1;
+  const int max_tiles = cdiv(p->chunk_tok, 64);
+  p->nsplit = 1;
+  if (p->n_seg > 0) {
+    const long long want = (kSplitTarget + BH * p->n_seg - 1) / (BH * p->n_seg);
+    p->nsplit = static_cast<int>(want < 1 ? 1 : (want > max_tiles ? max_tiles : want));
+  }
+  p->pairs = cdiv(cdiv(p->chunk_tok, 128), 2);
+  const long long units = BH * p->nc * static_cast<long long>(p->pairs);
+  if (units > INT_MAX || BH * p->n_seg * static_cast<long long>(p->nsplit) > INT_MAX) return REHYAT_EINVAL;
+  p->n_units = static_cast<int>(units);
+  const size_t D2 = 2 * static_cast<size_t>(d);
+  const size_t segs = static_cast<size_t>(BH) * p->n_seg * p->nsplit;
+  const size_t chunks = static_cast<size_t>(BH) * p->nc;
+  size_t off = 0;
+  p->off_pS = off; off += align256(segs * D2 * d * 4);
+  p->off_pz = off; off += align256(segs * D2 * 4);
+  p->off_hi = off; off += align256(chunks * D2 * d * 2);
+  p->off_lo = off; off += align256(chunks * D2 * d * 2);
+  p->off_zt = off; off += align256(chunks * D2 * 4);
+  p->bytes = off > 0 ? off : 256;
+  const size_t segs1 = static_cast<size_t>(BH) * p->n_seg;
+  off = 0;
+  p->f32_off_pS = off; off += align256(segs1 * D2 * d * 4);
+  p->f32_off_pz = off; off += align256(segs1 * D2 * 4);
+  p->f32_off_S = off; off += align256(chunks * D2 * d * 4);
+  p->f32_off_zt = off; off += align256(chunks * D2 * 4);
+  p->f32_bytes = off;
+  if (p->nc > 65535 || p->BH > 65535) p->f32_bytes = 0;  // fp32 grids use y/z dims
+  return REHYAT_OK;
+}
+
+struct StepPlan {
+  int BH, D, Nq, Nk, evict_tok, nsplit, pairs, n_units;
+  size_t off_hi, off_lo, off_pS, off_pz, bytes;
+  size_t f32_off_pS, f32_off_pz, f32_bytes;
+};
+
+int plan_step(int B, int H, int S_tok, int d, int qf, int cf, int ef, StepPlan* p) {
+  if (B < 1 || H < 1 || S_tok < 1 || qf < 1 || cf < 0 || ef < 0) return REHYAT_EINVAL;
+  int st = check_d(d);
+  if (st != REHYAT_OK) return st;
+  if (static_cast<long long>(ef) > static_cast<long long>(cf) + qf) return REHYAT_EINVAL;
+  const long long BH = static_cast<long long>(B) * H;
+  const long long Nq = static_cast<long long>(qf) * S_tok;
+  const long long Nk = (static_cast<long long>(cf) + qf) * S_tok;
+  if (BH > 65535 || Nk > INT_MAX / 2) return REHYAT_EINVAL;
+  if (BH * Nk * d > (1LL << 46)) return REHYAT_EINVAL;
+  p->BH = static_cast<int>(BH);
+  p->D = d;
+  p->Nq = static_cast<int>(Nq);
+  p->Nk = static_cast<int>(Nk);
+  p->evict_tok = ef * S_tok;
+  const int max_tiles = cdiv(p->evict_tok > 0 ? p->evict_tok : 1, 64);
+  const long long want = (kSplitTarget + BH - 1) / BH;
+  p->nsplit = static_cast<int>(want < 1 ? 1 : (want > max_tiles ? max_tiles : want));
+  p->pairs = cdiv(cdiv(p->Nq, 128), 2);
+  const long long units = BH * p->pairs;
+  if (units > INT_MAX) return REHYAT_EINVAL;
+  p->n_units = static_cast<int>(units);
+  const size_t D2 = 2 * static_cast<size_t>(d);
+  size_t off = 0;
+  p->off_hi = off; off += align256(static_cast<size_t>(BH) * D2 * d * 2);
+  p->off_lo = off; off += align256(static_cast<size_t>(BH) * D2 * d * 2);
+  p->off_pS = off; off += align256(static_cast<size_t>(BH) * p->nsplit * D2 * d * 4);
+  p->off_pz = off; off += align256(static_cast<size_t>(BH) * p->nsplit * D2 * 4);
+  p->bytes = off;
+  off = 0;
+  p->f32_off_pS = off; off += align256(static_cast<size_t>(BH) * D2 * d * 4);
+  p->f32_off_pz = off; off += align256(static_cast<size_t>(BH) * D2 * 4);
+  p->f32_bytes = off;
+  return REHYAT_OK;
+}
+
+// ---------------------------------------------------------------------------
+// TMA tensor maps (driver entry point fetched through the runtime, so the
+// library does not link libcuda directly)
+// ---------------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(f);
+  });
+  return fn;
+}
+
+// bf16 tensor [depth, rows, inner] (inner fastest), boxes of 64 x box_rows,
+// 128-byte swizzle, zero fill out of bounds.
+bool make_map(CUtensorMap* m, const void* base, long long inner, long long rows, long long depth, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(rows),
+                        static_cast<cuuint64_t>(depth)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(inner) * 2, static_cast<cuuint64_t>(inner) * 2 * rows};
+  cuuint32_t box[3] = {64u, static_cast<cuuint32_t>(box_rows), 1u};
+  cuuint32_t estr[3] = {1u, 1u, 1u};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int cuda_status(cudaError_t e) { return e == cudaSuccess ? REHYAT_OK : REHYAT_ECUDA; }
+
+// ---------------------------------------------------------------------------
+// stages
+// ---------------------------------------------------------------------------
+int run_states(const void* k, const void* v, const FwdPlan& P, uint8_t* ws, float* Sf_out, float* z_out,
+               cudaStream_t s) {
+  float* pS = reinterpret_cast<float*>(ws + P.off_pS);
+  float* pz = reinterpret_cast<float*>(ws + P.off_pz);
+  if (P.n_seg > 0) {
+    StateParams sp;
+    std::memset(&sp, 0, sizeof(sp));
+    if (!make_map(&sp.tm_k, k, P.D, P.N, P.BH, 64) || !make_map(&sp.tm_v, v, P.D, P.N, P.BH, 64))
+      return REHYAT_ECUDA;
+    sp.sg = SegGeom{P.N, P.chunk_tok, P.ovl_tok, P.n_seg, P.nsplit, 0, 0};
+    sp.BH = P.BH;
+    sp.part_S = pS;
+    sp.part_z = pz;
+    int st = cuda_status(launch_chunk_state(P.D, sp, P.BH * P.n_seg * P.nsplit, s));
+    if (st != REHYAT_OK) return st;
+  }
+  if (Sf_out != nullptr)
+    return cuda_status(launch_state_scan(pS, pz, P.BH, P.n_seg, P.nsplit, P.nc, P.D, nullptr, nullptr, Sf_out,
+                                         z_out, s));
+  return cuda_status(launch_state_scan(pS, pz, P.BH, P.n_seg, P.nsplit, P.nc, P.D,
+                                       reinterpret_cast<__nv_bfloat16*>(ws + P.off_hi),
+                                       reinterpret_cast<__nv_bfloat16*>(ws + P.off_lo), nullptr,
+                                       reinterpret_cast<float*>(ws + P.off_zt), s));
+}
+
+int run_attention(const void* q, const void* k, const void* v, const FwdPlan& P, uint8_t* ws, void* out,
+                  float* aS, float* nS, float* aL, float* nL, float* Mo, cudaStream_t s) {
+  AttnParams ap;
+  std::memset(&ap, 0, sizeof(ap));
+  if (!make_map(&ap.tm_q, q, P.D, P.N, P.BH, 128) || !make_map(&ap.tm_k, k, P.D, P.N, P.BH, 128) ||
+      !make_map(&ap.tm_v, v, P.D, P.N, P.BH, 128) ||
+      !make_map(&ap.tm_hi, ws + P.off_hi, P.D, 2LL * P.D, static_cast<long long>(P.BH) * P.nc, 128) ||
+      !make_map(&ap.tm_lo, ws + P.off_lo, P.D, 2LL * P.D, static_cast<long long>(P.BH) * P.nc, 128))
+    return REHYAT_ECUDA;
+  ap.g = ChunkGeom{P.N, P.N, P.chunk_tok, P.ovl_tok, P.nc, 0};
+  ap.BH = P.BH;
+  ap.pairs = P.pairs;
+  ap.state_mul = P.nc;
+  ap.scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(P.D));
+  ap.z = reinterpret_cast<const float*>(ws + P.off_zt);
+  ap.z_bh = 2LL * P.D * P.nc;
+  ap.z_t = 2LL * P.D;
+  ap.out = static_cast<__nv_bfloat16*>(out);
+  ap.aS = aS; ap.nS = nS; ap.aL = aL; ap.nL = nL; ap.Mo = Mo;
+  return cuda_status(launch_attention(P.D, aS != nullptr, ap, P.n_units, s));
+}
+
+struct WsGuard {  // stream-ordered scratch owned by one call
+  void* p = nullptr;
+  cudaStream_t s;
+  explicit WsGuard(cudaStream_t st) : s(st) {}
+  int alloc(size_t bytes) {
+    if (cudaMallocAsync(&p, bytes > 0 ? bytes : 256, s) != cudaSuccess) {
+      (void)cudaGetLastError();
+      p = nullptr;
+      return REHYAT_ENOMEM;
+    }
+    return REHYAT_OK;
+  }
+  ~WsGuard() {
+    if (p != nullptr) (void)cudaFreeAsync(p, s);
+  }
+};
+
+int check_qkvo(const void* q, const void* k, const void* v, const void* o) {
+  int st = check_ptr(q);
+  if (st == REHYAT_OK) st = check_ptr(k);
+  if (st == REHYAT_OK) st = check_ptr(v);
+  if (st == REHYAT_OK) st = check_ptr(o);
+  return st;
+}
+
+}  // namespace
+
+// ===========================================================================
+// exported entry points
+// ===========================================================================
+REHYAT_API const char* rehyat_status_string(int status) {
+  switch (status) {
+    case REHYAT_OK: return "REHYAT_OK";
+    case REHYAT_EINVAL: return "REHYAT_EINVAL: invalid argument";
+    case REHYAT_EUNSUPPORTED: return "REHYAT_EUNSUPPORTED: unsupported configuration (d must be 64 or 128)";
+    case REHYAT_ENOMEM: return "REHYAT_ENOMEM: workspace allocation failed or workspace too small";
+    case REHYAT_ECUDA: return "REHYAT_ECUDA: CUDA call or kernel launch failed";
+    case REHYAT_ETIMEOUT: return "REHYAT_ETIMEOUT: a bounded device-side wait ran out";
+    default: return "REHYAT_UNKNOWN_STATUS";
+  }
+}
+
+REHYAT_API int rehyat_forward_workspace_bytes(int B, int H, int F, int S_tok, int d, int chunk_frames,
+                                              int overlap_frames, size_t* bytes) {
+  if (bytes == nullptr) return REHYAT_EINVAL;
+  FwdPlan P;
+  int st = plan_forward(B, H, F, S_tok, d, chunk_frames, overlap_frames, &P);
+  if (st != REHYAT_OK) return st;
+  *bytes = P.bytes;
+  return REHYAT_OK;
+}
+
+REHYAT_API int rehyat_forward_states(const void* k, const void* v, int B, int H, int F, int S_tok, int d,
+                                     int chunk_frames, int overlap_frames, void* workspace,
+                                     size_t workspace_bytes, void* stream) {
+  FwdPlan P;
+  int st = plan_forward(B, H, F, S_tok, d, chunk_frames, overlap_frames, &P);
+  if (st != REHYAT_OK) return st;
+  if (check_ptr(k) || check_ptr(v) || check_ptr(workspace)) return REHYAT_EINVAL;
+  if (reinterpret_cast<uintptr_t>(workspace) % 256 != 0) return REHYAT_EINVAL;
+  if (workspace_bytes < P.bytes) return REHYAT_ENOMEM;
+  return run_states(k, v, P, static_cast<uint8_t*>(workspace), nullptr, nullptr, static_cast<cudaStream_t>(stream));
+}
+
+REHYAT_API int rehyat_forward_attention(const void* q, const void* k, const void* v, int B, int H, int F,
+                                        int S_tok, int d, int chunk_frames, int overlap_frames, void* out,
+                                        void* workspace, size_t workspace_bytes, void* stream) {
+  FwdPlan P;
+  int st = plan_forward(B, H, F, S_tok, d, chunk_frames, overlap_frames, &P);
+  if (st != REHYAT_OK) return st;
+  if (check_qkvo(q, k, v, out) || check_ptr(workspace)) return REHYAT_EINVAL;
+  if (reinterpret_cast<uintptr_t>(workspace) % 256 != 0) return REHYAT_EINVAL;
+  if (workspace_bytes < P.bytes) return REHYAT_ENOMEM;
+  return run_attention(q, k, v, P, static_cast<uint8_t*>(workspace), out, nullptr, nullptr, nullptr, nullptr,
+                       nullptr, static_cast<cudaStream_t>(stream));
+}
+
+REHYAT_API int rehyat_forward_ws(const void* q, const void* k, const void* v, int B, int H, int F, int S_tok,
+                                 int d, int chunk_frames, int overlap_frames, void* out, void* workspace,
+                                 size_t workspace_bytes, void* stream) {
+  int st = rehyat_forward_states(k, v, B, H, F, S_tok, d, chunk_frames, overlap_frames, workspace,
+                                 workspace_bytes, stream);
+  if (st != REHYAT_OK) return st;
+  return rehyat_forward_attention(q, k, v, B, H, F, S_tok, d, chunk_frames, overlap_frames, out, workspace,
+                                  workspace_bytes, stream);
+}
+
+REHYAT_API int rehyat_forward(const void* q, const void* k, const void* v, int B, int H, int F, int S_tok, int d,
+                              int chunk_frames, int overlap_frames, void* out, void* stream) {
+  FwdPlan P;
+  int st = plan_forward(B, H, F, S_tok, d, chunk_frames, overlap_frames, &P);
+  if (st != REHYAT_OK) return st;
+  if (check_qkvo(q, k, v, out)) return REHYAT_EINVAL;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  WsGuard ws(s);
+  st = ws.alloc(P.bytes);
+  if (st != REHYAT_OK) return st;
+  return rehyat_forward_ws(q, k, v, B, H, F, S_tok, d, chunk_frames, overlap_frames, out, ws.p, P.bytes, stream);
+}
+
+REHYAT_API int rehyat_forward_parts(const void* q, const void* k, const void* v, int B, int H, int F, int S_tok,
+                                    int d, int chunk_frames, int overlap_frames, float* aS, float* nS, float* aL,
+                                    float* nL, float* M, void* stream) {
+  FwdPlan P;
+  int st = plan_forward(B, H, F, S_tok, d, chunk_frames, overlap_frames, &P);
+  if (st != REHYAT_OK) return st;
+  if (check_ptr(q) || check_ptr(k) || check_ptr(v) || check_ptr(aS) || check_ptr(aL) || nS == nullptr ||
+      nL == nullptr || M == nullptr)
+    return REHYAT_EINVAL;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  WsGuard ws(s);
+  st = ws.alloc(P.bytes);
+  if (st != REHYAT_OK) return st;
+  uint8_t* w = static_cast<uint8_t*>(ws.p);
+  st = run_states(k, v, P, w, nullptr, nullptr, s);
+  if (st != REHYAT_OK) return st;
+  return run_attention(q, k, v, P, w, nullptr, aS, nS, aL, nL, M, s);
+}
+
+REHYAT_API int rehyat_chunk_states(const void* k, const void* v, int B, int H, int F, int S_tok, int d,
+                                   int chunk_frames, int overlap_frames, float* S, float* z, void* stream) {
+  FwdPlan P;
+  int st = plan_forward(B, H, F, S_tok, d, chunk_frames, overlap_frames, &P);
+  if (st != REHYAT_OK) return st;
+  if (check_ptr(k) || check_ptr(v) || S == nullptr || z == nullptr) return REHYAT_EINVAL;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  WsGuard ws(s);
+  st = ws.alloc(P.off_hi);  // partials only
+  if (st != REHYAT_OK) return st;
+  return run_states(k, v, P, static_cast<uint8_t*>(ws.p), S, z, s);
+}
+
+REHYAT_API int rehyat_forward_f32(const float* q, const float* k, const float* v, int B, int H, int F, int S_tok,
+                                  int d, int chunk_frames, int overlap_frames, float* out, void* stream) {
+  FwdPlan P;
+  int st = plan_forward(B, H, F, S_tok, d, chunk_frames, overlap_frames, &P);
+  if (st != REHYAT_OK) return st;
+  if (P.f32_bytes == 0) return REHYAT_EINVAL;
+  if (check_qkvo(q, k, v, out)) return REHYAT_EINVAL;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  WsGuard ws(s);
+  st = ws.alloc(P.f32_bytes);
+  if (st != REHYAT_OK) return st;
+  uint8_t* w = static_cast<uint8_t*>(ws.p);
+  float* pS = reinterpret_cast<float*>(w + P.f32_off_pS);
+  float* pz = reinterpret_cast<float*>(w + P.f32_off_pz);
+  float* Sf = reinterpret_cast<float*>(w + P.f32_off_S);
+  float* zt = reinterpret_cast<float*>(w + P.f32_off_zt);
+  StateF32Params sp;
+  sp.sg = SegGeom{P.N, P.chunk_tok, P.ovl_tok, P.n_seg, 1, 0, 0};
+  sp.BH = P.BH;
+  sp.D = P.D;
+  sp.k = k;
+  sp.v = v;
+  sp.part_S = pS;
+  sp.part_z = pz;
+  st = cuda_status(launch_chunk_state_f32(sp, s));
+  if (st != REHYAT_OK) return st;
+  st = cuda_status(launch_state_scan(pS, pz, P.BH, P.n_seg, 1, P.nc, P.D, nullptr, nullptr, Sf, zt, s));
+  if (st != REHYAT_OK) return st;
+  AttnF32Params ap;
+  ap.g = ChunkGeom{P.N, P.N, P.chunk_tok, P.ovl_tok, P.nc, 0};
+  ap.BH = P.BH;
+  ap.D = P.D;
+  ap.q = q; ap.k = k; ap.v = v;
+  ap.S = Sf;
+  ap.S_bh = 2LL * P.D * P.D * P.nc;
+  ap.S_t = 2LL * P.D * P.D;
+  ap.z = zt;
+  ap.z_bh = 2LL * P.D * P.nc;
+  ap.z_t = 2LL * P.D;
+  ap.out = out;
+  return cuda_status(launch_attention_f32(ap, P.nc, s));
+}
+
+// ---------------------------------------------------------------------------
+// recurrent form
+// ---------------------------------------------------------------------------
+REHYAT_API int rehyat_step_workspace_bytes(int B, int H, int S_tok, int d, int q_frames, int ctx_frames,
+                                           int evict_frames, size_t* bytes) {
+  if (bytes == nullptr) return REHYAT_EINVAL;
+  StepPlan P;
+  int st = plan_step(B, H, S_tok, d, q_frames, ctx_frames, evict_frames, &P);
+  if (st != REHYAT_OK) return st;
+  *bytes = P.bytes;
+  return REHYAT_OK;
+}
+
+REHYAT_API int rehyat_step_ws(const void* q_c, const void* k_c, const void* v_c, float* state_S, float* state_z,
+                              void* out_c, int B, int H, int S_tok, int d, int q_frames, int ctx_frames,
+                              int evict_frames, void* workspace, size_t workspace_bytes, void* stream) {
+  StepPlan P;
+  int st = plan_step(B, H, S_tok, d, q_frames, ctx_frames, evict_frames, &P);
+  if (st != REHYAT_OK) return st;
+  if (check_qkvo(q_c, k_c, v_c, out_c) || check_ptr(state_S) || check_ptr(state_z) || check_ptr(workspace))
+    return REHYAT_EINVAL;
+  if (reinterpret_cast<uintptr_t>(workspace) % 256 != 0) return REHYAT_EINVAL;
+  if (workspace_bytes < P.bytes) return REHYAT_ENOMEM;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* w = static_cast<uint8_t*>(workspace);
+  __nv_bfloat16* hi = reinterpret_cast<__nv_bfloat16*>(w + P.off_hi);
+  __nv_bfloat16* lo = reinterpret_cast<__nv_bfloat16*>(w + P.off_lo);
+  st = cuda_status(launch_state_split(state_S, static_cast<long long>(P.BH) * 2 * P.D * P.D, hi, lo, s));
+  if (st != REHYAT_OK) return st;
+  AttnParams ap;
+  std::memset(&ap, 0, sizeof(ap));
+  if (!make_map(&ap.tm_q, q_c, P.D, P.Nq, P.BH, 128) || !make_map(&ap.tm_k, k_c, P.D, P.Nk, P.BH, 128) ||
+      !make_map(&ap.tm_v, v_c, P.D, P.Nk, P.BH, 128) || !make_map(&ap.tm_hi, hi, P.D, 2LL * P.D, P.BH, 128) ||
+      !make_map(&ap.tm_lo, lo, P.D, 2LL * P.D, P.BH, 128))
+    return REHYAT_ECUDA;
+  ap.g = ChunkGeom{P.Nq, P.Nk, P.Nq, 0, 1, 1};
+  ap.BH = P.BH;
+  ap.pairs = P.pairs;
+  ap.state_mul = 1;
+  ap.scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(P.D));
+  ap.z = state_z;
+  ap.z_bh = 2LL * P.D;
+  ap.z_t = 0;
+  ap.out = static_cast<__nv_bfloat16*>(out_c);
+  st = cuda_status(launch_attention(P.D, false, ap, P.n_units, s));
+  if (st != REHYAT_OK || P.evict_tok == 0) return st;
+  StateParams sp;
+  std::memset(&sp, 0, sizeof(sp));
+  if (!make_map(&sp.tm_k, k_c, P.D, P.Nk, P.BH, 64) || !make_map(&sp.tm_v, v_c, P.D, P.Nk, P.BH, 64))
+    return REHYAT_ECUDA;
+  sp.sg = SegGeom{P.Nk, 0, 0, 1, P.nsplit, 1, P.evict_tok};
+  sp.BH = P.BH;
+  sp.part_S = reinterpret_cast<float*>(w + P.off_pS);
+  sp.part_z = reinterpret_cast<float*>(w + P.off_pz);
+  st = cuda_status(launch_chunk_state(P.D, sp, P.BH * P.nsplit, s));
+  if (st != REHYAT_OK) return st;
+  return cuda_status(launch_state_accumulate(sp.part_S, sp.part_z, P.BH, P.nsplit, P.D, state_S, state_z, s));
+}
+
+REHYAT_API int rehyat_step(const void* q_c, const void* k_c, const void* v_c, float* state_S, float* state_z,
+                           void* out_c, int B, int H, int S_tok, int d, int q_frames, int ctx_frames,
+                           int evict_frames, void* stream) {
+  StepPlan P;
+  int st = plan_step(B, H, S_tok, d, q_frames, ctx_frames, evict_frames, &P);
+  if (st != REHYAT_OK) return st;
+  if (check_qkvo(q_c, k_c, v_c, out_c) || check_ptr(state_S) || check_ptr(state_z)) return REHYAT_EINVAL;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  WsGuard ws(s);
+  st = ws.alloc(P.bytes);
+  if (st != REHYAT_OK) return st;
+  return rehyat_step_ws(q_c, k_c, v_c, state_S, state_z, out_c, B, H, S_tok, d, q_frames, ctx_frames,
+                        evict_frames, ws.p, P.bytes, stream);
+}
+
+REHYAT_API int rehyat_step_f32(const float* q_c, const float* k_c, const float* v_c, float* state_S,
+                               float* state_z, float* out_c, int B, int H, int S_tok, int d, int q_frames,
+                               int ctx_frames, int evict_frames, void* stream) {
+  StepPlan P;
+  int st = plan_step(B, H, S_tok, d, q_frames, ctx_frames, evict_frames, &P);
+  if (st != REHYAT_OK) return st;
+  if (check_qkvo(q_c, k_c, v_c, out_c) || check_ptr(state_S) || check_ptr(state_z)) return REHYAT_EINVAL;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  AttnF32Params ap;
+  ap.g = ChunkGeom{P.Nq, P.Nk, P.Nq, 0, 1, 1};
+  ap.BH = P.BH;
+  ap.D = P.D;
+  ap.q = q_c; ap.k = k_c; ap.v = v_c;
+  ap.S = state_S;
+  ap.S_bh = 2LL * P.D * P.D;
+  ap.S_t = 0;
+  ap.z = state_z;
+  ap.z_bh = 2LL * P.D;
+  ap.z_t = 0;
+  ap.out = out_c;
+  st = cuda_status(launch_attention_f32(ap, 1, s));
+  if (st != REHYAT_OK || P.evict_tok == 0) return st;
+  WsGuard ws(s);
+  st = ws.alloc(P.f32_bytes);
+  if (st != REHYAT_OK) return st;
+  uint8_t* w = static_cast<uint8_t*>(ws.p);
+  StateF32Params sp;
+  sp.sg = SegGeom{P.Nk, 0, 0, 1, 1, 1, P.evict_tok};
+  sp.BH = P.BH;
+  sp.D = P.D;
+  sp.k = k_c;
+  sp.v = v_c;
+  sp.part_S = reinterpret_cast<float*>(w + P.f32_off_pS);
+  sp.part_z = reinterpret_cast<float*>(w + P.f32_off_pz);
+  st = cuda_status(launch_chunk_state_f32(sp, s));
+  if (st != REHYAT_OK) return st;
+  return cuda_status(launch_state_accumulate(sp.part_S, sp.part_z, P.BH, 1, P.D, state_S, state_z, s));
+}
+
+// ---------------------------------------------------------------------------
+// feature map, status
+// ---------------------------------------------------------------------------
+REHYAT_API int rehyat_phi(const void* x, int x_dtype, void* y, int y_dtype, int64_t rows, int d, void* stream) {
+  if (x == nullptr || y == nullptr || rows < 1 || d < 1) return REHYAT_EINVAL;
+  if ((x_dtype != REHYAT_DTYPE_BF16 && x_dtype != REHYAT_DTYPE_F32) ||
+      (y_dtype != REHYAT_DTYPE_BF16 && y_dtype != REHYAT_DTYPE_F32))
+    return REHYAT_EINVAL;
+  if (rows > (1LL << 40) / d) return REHYAT_EINVAL;
+  return cuda_status(launch_phi(x, x_dtype == REHYAT_DTYPE_F32, y, y_dtype == REHYAT_DTYPE_F32, rows, d,
+                                static_cast<cudaStream_t>(stream)));
+}
+
+REHYAT_API int rehyat_device_status(unsigned int* detail) {
+  unsigned int v = 0;
+  if (cudaDeviceSynchronize() != cudaSuccess) return REHYAT_ECUDA;
+  if (read_and_clear_device_error(&v) != cudaSuccess) return REHYAT_ECUDA;
+  if (detail != nullptr) *detail = v;
+  return v == 0 ? REHYAT_OK : REHYAT_ETIMEOUT;
+}

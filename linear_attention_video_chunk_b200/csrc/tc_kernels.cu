@@ -1,0 +1,845 @@
+// tc_kernels.cu -- tensor-core (tcgen05 / TMEM / TMA) kernels for sm_100a.
+//
+// 1. hybrid_chunk_attn_kernel: the fused per-chunk hybrid attention of
+//    "ReHyAt: Recurrent Hybrid Attention for Video Diffusion Transformers",
+//    §3.2 (joint normaliser y = (a^S + a^L) / (n^S + n^L)) over the §3.3
+//    sets: exact softmax over the chunk's window [lo_t, hi_t) plus the linear
+//    term phi(q) S_t, phi(q) z_t of every earlier key (§3.1 caching).
+// 2. phi_state_kernel: phi(K)^T V and sum phi(K) per key segment (the two
+//    query-independent sums of §3.1), phi of §3.2 with P = 2, psi = 1 + elu.
+//
+// Layout conventions (all operand tiles use the 128-byte TMA swizzle):
+//   a "box" is 128 B wide (64 bf16) and R rows tall; row r lives at r*128 and
+//   its 16-byte chunk c at ((c ^ (r & 7)) * 16).  A D-wide tile is D/64 boxes.
+#include <cstdint>
+
+#include "kernels.cuh"
+#include "ptx.cuh"
+
+namespace rehyat {
+namespace {
+
+constexpr uint32_t kFull = 0xffffffffu;
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+
+// Bounded warp-wide wait: every lane polls; the result is uniform.
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int* abort) {
+  const bool ok = mbar_wait(bar, parity, abort);
+  return __all_sync(kFull, ok);
+}
+
+// Bounded wait that ignores the abort word: used to drain in-flight async
+// work (TMA copies, MMAs) before a CTA releases its shared / tensor memory.
+__device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity) {
+  volatile int never = 0;
+  (void)mbar_wait(bar, parity, &never);
+}
+
+__device__ __forceinline__ float psi1(float x) {  // 1 + elu(x)
+  return x > 0.f ? x + 1.f : ex2(x * kLog2e);
+}
+
+// ============================================================================
+// Fused chunk attention
+// ============================================================================
+template <int D>
+struct AttnCfg {
+  static constexpr int NBOX = D / 64;
+  static constexpr int BOX_BYTES = 128 * 128;               // 128 rows x 128 B
+  static constexpr int TILE_BYTES = NBOX * BOX_BYTES;       // 128 x D bf16
+  static constexpr int NSLOTS = (D == 128) ? 5 : 8;         // K/V/state ring
+  static constexpr int SPP = (2 * D) / 128;                 // state slots per hi|lo part
+  static constexpr int OFF_RING = 0;                        // ring first, then the Q tiles:
+  static constexpr int OFF_Q = NSLOTS * TILE_BYTES;         // operand reads stay inside the
+  static constexpr int OFF_BAR = OFF_Q + 2 * TILE_BYTES;    // data area whatever the layout
+  static constexpr int SMEM = OFF_BAR + 512 + 1024;         // + barriers, + alignment slack
+  // barrier indices
+  static constexpr int B_Q = 0;
+  static constexpr int B_FULL = 1;
+  static constexpr int B_EMPTY = B_FULL + NSLOTS;
+  static constexpr int B_S = B_EMPTY + NSLOTS;   // [2] scores ready in TMEM
+  static constexpr int B_P = B_S + 2;            // [2] probabilities written to TMEM
+  static constexpr int B_O = B_P + 2;            // [2] last P.V done
+  static constexpr int B_PHI = B_O + 2;          // [2] scaled phi(Q) written to TMEM
+  static constexpr int B_LIN = B_PHI + 2;        // [2] linear MMA done
+  static constexpr int B_FIN = B_LIN + 2;        // MMA drain
+  static constexpr int NBARS = B_FIN + 1;
+  static_assert(NBARS * 8 <= 256, "barrier area");
+  static_assert(SMEM <= 232448, "shared memory");
+  // TMEM columns: S/P of tile X at X*128, O of tile X at 256 + X*D.
+  static constexpr uint32_t TMEM_COLS = 512;
+  static constexpr uint32_t IDESC_S = idesc_bf16_f32(128, 128, 0, 0);  // Q K^T: both K-major
+  static constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, D, 0, 1);   // P V, phi~ S: B MN-major
+};
+
+template <int D, bool PARTS>
+__global__ void __launch_bounds__(320, 1) hybrid_chunk_attn_kernel(const __grid_constant__ AttnParams p) {
+  using C = AttnCfg<D>;
+  constexpr int NS = C::NSLOTS;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  // ---- unit -> (bh, chunk t, pair of 128-row query tiles) -----------------
+  // Chunks are visited 1, 2, ..., n-1, 0: chunk 0 has no overlap frames (the
+  // shortest window), so the longest units start first.
+  const int u = blockIdx.x;
+  const int pair = u % p.pairs;
+  const int rest = u / p.pairs;
+  const int bh = rest % p.BH;
+  const int o = rest / p.BH;
+  const int t = (p.g.n_chunks > 1) ? (o + 1) % p.g.n_chunks : 0;
+  int q0, q1, lo, hi;
+  p.g.chunk(t, q0, q1, lo, hi);
+  const int rowA0 = q0 + pair * 256;
+  const int rowB0 = rowA0 + 128;
+  const int nA = imin(imax(q1 - rowA0, 0), 128);
+  const int nB = imin(imax(q1 - rowB0, 0), 128);
+  if (nA <= 0) return;  // the ragged last chunk has fewer tiles (uniform exit)
+  const bool hasB = nB > 0;
+  const int win = hi - lo;  // >= 1
+  const int ntiles = cdiv(win, 128);
+
+  uint8_t* barea = smem + C::OFF_BAR;
+  const uint32_t bar0 = smem_u32(barea);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(barea + 256);
+  volatile int* abort = reinterpret_cast<volatile int*>(barea + 260);
+  int* lin_flag = reinterpret_cast<int*>(barea + 264);
+#define BAR(i) (bar0 + 8u * static_cast<uint32_t>(i))
+
+  if (threadIdx.x == 0) {
+    mbar_init(BAR(C::B_Q), 1);
+    for (int i = 0; i < NS; ++i) {
+      mbar_init(BAR(C::B_FULL + i), 1);
+      mbar_init(BAR(C::B_EMPTY + i), 1);
+    }
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(BAR(C::B_S + x), 1);
+      mbar_init(BAR(C::B_P + x), 128);
+      mbar_init(BAR(C::B_O + x), 1);
+      mbar_init(BAR(C::B_PHI + x), 128);
+      mbar_init(BAR(C::B_LIN + x), 1);
+    }
+    mbar_init(BAR(C::B_FIN), 1);
+    *abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    // The linear set is non-empty iff z_t > 0 somewhere (phi > 0 elementwise).
+    int f = 0;
+    if (p.z != nullptr) {
+      const float* zp = p.z + bh * p.z_bh + t * p.z_t;
+      for (int e = lane; e < 2 * D; e += 32) f |= (zp[e] > 0.f) ? 1 : 0;
+    }
+    f = __any_sync(kFull, f);
+    if (lane == 0) *lin_flag = f;
+  }
+  if (warp == 8 && lane == 0) {
+    prefetch_tmap(&p.tm_q);
+    prefetch_tmap(&p.tm_k);
+    prefetch_tmap(&p.tm_v);
+  }
+  if (warp == 9) {
+    tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const bool has_lin = (*lin_flag) != 0;
+
+  if (warp < 8) {
+    // ======================= softmax / epilogue warps =======================
+    const int X = warp >> 2;  // query tile A (0) or B (1)
+    const int wl = warp & 3;  // TMEM lane quarter
+    const int nX = X ? nB : nA;
+    if (X == 0 || hasB) {
+      const int r = wl * 32 + lane;  // row inside the 128-row tile
+      const uint32_t lane_off = static_cast<uint32_t>(wl * 32) << 16;
+      const uint32_t tS = tmem + lane_off + X * 128;
+      const uint32_t tO = tmem + lane_off + 256 + X * D;
+      // Running shift (log2 units).  With a non-empty linear set it starts
+      // at 0, so the final shift M = max(m, 0) keeps exp(-M) <= 1 on the
+      // linear terms; without one it is the usual running maximum.
+      float m_used = has_lin ? 0.f : -INFINITY;
+      float l = 0.f;
+      bool ok = true;
+      for (int j = 0; j < ntiles; ++j) {
+        ok = warp_wait(BAR(C::B_S + X), j & 1, abort);
+        if (!ok) break;
+        tc_fence_after();
+        uint32_t s[4][32];
+        tmem_ld32(tS + 0, s[0]);
+        tmem_ld32(tS + 32, s[1]);
+        tmem_ld32(tS + 64, s[2]);
+        tmem_ld32(tS + 96, s[3]);
+        tmem_ld_wait();
+        reg_fence(s[0]);
+        reg_fence(s[1]);
+        reg_fence(s[2]);
+        reg_fence(s[3]);
+        const int valid = win - j * 128;  // keys of this tile inside the window
+        float mx = -INFINITY;
+#pragma unroll
+        for (int a = 0; a < 4; ++a) {
+#pragma unroll
+          for (int c = 0; c < 32; ++c) {
+            float x = __uint_as_float(s[a][c]) * p.scale_log2;
+            x = (a * 32 + c < valid) ? x : -INFINITY;
+            s[a][c] = __float_as_uint(x);
+            mx = fmaxf(mx, x);
+          }
+        }
+        // Lazy rescaling: move the shift only when the row maximum exceeds
+        // it by more than 2^8, so P <= 256 and fp32 sums stay exact enough.
+        const bool need = mx > m_used + 8.f;
+        const bool warp_need = __any_sync(kFull, need) != 0;
+        const float mnew = need ? mx : m_used;
+        const float alpha = need ? ex2(m_used - mnew) : 1.f;
+        m_used = mnew;
+        float rs = 0.f;
+        uint32_t pk[2][32];
+#pragma unroll
+        for (int a = 0; a < 4; ++a) {
+#pragma unroll
+          for (int c = 0; c < 16; ++c) {
+            const float p0 = ex2(__uint_as_float(s[a][2 * c]) - m_used);
+            const float p1 = ex2(__uint_as_float(s[a][2 * c + 1]) - m_used);
+            rs += p0 + p1;
+            pk[a >> 1][(a & 1) * 16 + c] = pack_bf16(p0, p1);
+          }
+        }
+        l = l * alpha + rs;
+        // P (bf16, two per column) overwrites the first 64 columns of S.
+        tmem_st32(tS + 0, pk[0]);
+        tmem_st32(tS + 32, pk[1]);
+        if (warp_need && j > 0) {
+          // O holds tiles 0..j-1 (their P.V completed before S_j was
+          // signalled) and must move to the new shift before P_j.V_j.
+#pragma unroll
+          for (int a = 0; a < D / 32; ++a) {
+            uint32_t ov[32];
+            tmem_ld32(tO + 32 * a, ov);
+            tmem_ld_wait();
+            reg_fence(ov);
+#pragma unroll
+            for (int c = 0; c < 32; ++c) ov[c] = __float_as_uint(__uint_as_float(ov[c]) * alpha);
+            tmem_st32(tO + 32 * a, ov);
+          }
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(BAR(C::B_P + X));
+      }
+
+      if (ok) ok = warp_wait(BAR(C::B_O + X), 0, abort);
+      tc_fence_after();
+      const bool vrow = r < nX;
+      const size_t grow = static_cast<size_t>(bh) * p.g.N_q + (X ? rowB0 : rowA0) + r;
+
+      if (PARTS && ok) {
+#pragma unroll
+        for (int a = 0; a < D / 32; ++a) {
+          uint32_t ov[32];
+          tmem_ld32(tO + 32 * a, ov);
+          tmem_ld_wait();
+          reg_fence(ov);
+          if (vrow) {
+            float4* dst = reinterpret_cast<float4*>(p.aS + grow * D + 32 * a);
+#pragma unroll
+            for (int c = 0; c < 8; ++c)
+              dst[c] = make_float4(__uint_as_float(ov[4 * c]), __uint_as_float(ov[4 * c + 1]),
+                                   __uint_as_float(ov[4 * c + 2]), __uint_as_float(ov[4 * c + 3]));
+          }
+        }
+        if (vrow) {
+          p.nS[grow] = l;
+          p.Mo[grow] = m_used * kLn2;
+        }
+      }
+
+      // ---- linear term: phi(q) S_t and phi(q) z_t (§3.1 cached sums) ----
+      float nl = 0.f, sc = 0.f;
+      if (has_lin && ok) {
+        sc = ex2(-m_used);  // exp(-M), <= 1
+        const float* zp = p.z + bh * p.z_bh + t * p.z_t;
+        const uint8_t* qrow = smem + C::OFF_Q + X * C::TILE_BYTES + r * 128;
+#pragma unroll
+        for (int b = 0; b < C::NBOX; ++b) {
+          uint32_t pa[32], pb[32];
+#pragma unroll
+          for (int cc = 0; cc < 8; ++cc) {
+            const uint4 raw =
+                *reinterpret_cast<const uint4*>(qrow + b * C::BOX_BYTES + ((cc ^ (r & 7)) << 4));
+            const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+              const float s0 = psi1(bf16lo(w[h]));
+              const float s1 = psi1(bf16hi(w[h]));
+              const int dim = 64 * b + 8 * cc + 2 * h;
+              nl += s0 * zp[dim] + (s0 * s0) * zp[D + dim] + s1 * zp[dim + 1] +
+                    (s1 * s1) * zp[D + dim + 1];
+              pa[cc * 4 + h] = pack_bf16(s0 * sc, s1 * sc);
+              pb[cc * 4 + h] = pack_bf16((s0 * s0) * sc, (s1 * s1) * sc);
+            }
+          }
+          // features psi (0..D-1) then psi^2 (D..2D-1), two per column
+          tmem_st32(tS + 32 * b, pa);
+          tmem_st32(tS + D / 2 + 32 * b, pb);
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(BAR(C::B_PHI + X));
+        ok = warp_wait(BAR(C::B_LIN + X), 0, abort);
+        tc_fence_after();
+      }
+
+      if (ok) {
+        if (!PARTS) {
+          const float inv = 1.f / (l + (has_lin ? nl * sc : 0.f));
+#pragma unroll
+          for (int a = 0; a < D / 32; ++a) {
+            uint32_t ov[32];
+            tmem_ld32(tO + 32 * a, ov);
+            tmem_ld_wait();
+            reg_fence(ov);
+            if (vrow) {
+              uint4* dst = reinterpret_cast<uint4*>(p.out + grow * D + 32 * a);
+#pragma unroll
+              for (int c = 0; c < 4; ++c) {
+                uint4 w;
+                w.x = pack_bf16(__uint_as_float(ov[8 * c + 0]) * inv, __uint_as_float(ov[8 * c + 1]) * inv);
+                w.y = pack_bf16(__uint_as_float(ov[8 * c + 2]) * inv, __uint_as_float(ov[8 * c + 3]) * inv);
+                w.z = pack_bf16(__uint_as_float(ov[8 * c + 4]) * inv, __uint_as_float(ov[8 * c + 5]) * inv);
+                w.w = pack_bf16(__uint_as_float(ov[8 * c + 6]) * inv, __uint_as_float(ov[8 * c + 7]) * inv);
+                dst[c] = w;
+              }
+            }
+          }
+        } else {
+#pragma unroll
+          for (int a = 0; a < D / 32; ++a) {
+            uint32_t ov[32];
+            if (has_lin) {
+              tmem_ld32(tO + 32 * a, ov);
+              tmem_ld_wait();
+              reg_fence(ov);
+            } else {
+#pragma unroll
+              for (int c = 0; c < 32; ++c) ov[c] = 0u;
+            }
+            if (vrow) {
+              float4* dst = reinterpret_cast<float4*>(p.aL + grow * D + 32 * a);
+#pragma unroll
+              for (int c = 0; c < 8; ++c)
+                dst[c] = make_float4(__uint_as_float(ov[4 * c]), __uint_as_float(ov[4 * c + 1]),
+                                     __uint_as_float(ov[4 * c + 2]), __uint_as_float(ov[4 * c + 3]));
+            }
+          }
+          if (vrow) p.nL[grow] = has_lin ? nl * sc : 0.f;
+        }
+      }
+    }
+  } else if (warp == 8) {
+    // =============================== TMA producer ============================
+    if (lane == 0) {
+      const uint32_t sq = smem_u32(smem + C::OFF_Q);
+      const uint32_t ring = smem_u32(smem + C::OFF_RING);
+      mbar_arrive_expect_tx(BAR(C::B_Q), (hasB ? 2 : 1) * C::TILE_BYTES);
+      for (int b = 0; b < C::NBOX; ++b) tma_load_3d(sq + b * C::BOX_BYTES, &p.tm_q, BAR(C::B_Q), 64 * b, rowA0, bh);
+      if (hasB)
+        for (int b = 0; b < C::NBOX; ++b)
+          tma_load_3d(sq + C::TILE_BYTES + b * C::BOX_BYTES, &p.tm_q, BAR(C::B_Q), 64 * b, rowB0, bh);
+      uint32_t seq = 0;
+      bool ok = true;
+      auto load_tile = [&](const CUtensorMap* tm, int y, int zc) {
+        const uint32_t slot = seq % NS;
+        ok = ok && mbar_wait(BAR(C::B_EMPTY + slot), ((seq / NS) & 1) ^ 1, abort);
+        if (!ok) return;
+        mbar_arrive_expect_tx(BAR(C::B_FULL + slot), C::TILE_BYTES);
+        for (int b = 0; b < C::NBOX; ++b)
+          tma_load_3d(ring + slot * C::TILE_BYTES + b * C::BOX_BYTES, tm, BAR(C::B_FULL + slot), 64 * b, y, zc);
+        ++seq;
+      };
+      for (int j = 0; j < ntiles && ok; ++j) {
+        load_tile(&p.tm_k, lo + 128 * j, bh);
+        load_tile(&p.tm_v, lo + 128 * j, bh);
+      }
+      if (has_lin) {
+        const int zc = bh * p.state_mul + (p.g.step ? 0 : t);
+        for (int part = 0; part < 2 && ok; ++part)
+          for (int rr = 0; rr < C::SPP && ok; ++rr) load_tile(part ? &p.tm_lo : &p.tm_hi, 128 * rr, zc);
+      }
+      // drain: every copy issued must have landed before the CTA exits
+      drain_wait(BAR(C::B_Q), 0);
+      for (uint32_t s2 = (seq > NS ? seq - NS : 0); s2 < seq; ++s2) drain_wait(BAR(C::B_FULL + s2 % NS), (s2 / NS) & 1);
+    }
+  } else {
+    // =============================== MMA issuer ==============================
+    if (lane == 0) {
+      const uint32_t qA = smem_u32(smem + C::OFF_Q);
+      const uint32_t qB = qA + C::TILE_BYTES;
+      const uint32_t ring = smem_u32(smem + C::OFF_RING);
+      auto slot_addr = [&](uint32_t sq) { return ring + (sq % NS) * C::TILE_BYTES; };
+      // Q K^T: A = Q tile, B = K tile, both K-major; K-step kk moves 32 B
+      // inside a 128-B swizzle row (box kk/4).
+      auto issue_S = [&](uint32_t d_tmem, uint32_t qa, uint32_t kb) {
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * C::BOX_BYTES + (kk & 3) * 32;
+          mma_ss(d_tmem, smem_desc_sw128(qa + off, 16, 1024), smem_desc_sw128(kb + off, 16, 1024),
+                 C::IDESC_S, kk > 0 ? 1u : 0u);
+        }
+      };
+      // P V: A = P in TMEM (8 columns per 16 keys), B = V tile MN-major:
+      // 16 keys = 2048 B; the two 64-column boxes are BOX_BYTES apart.
+      auto issue_PV = [&](uint32_t d_tmem, uint32_t a_tmem, uint32_t vb, bool first) {
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ts(d_tmem, a_tmem + kk * 8, smem_desc_sw128(vb + kk * 2048, C::BOX_BYTES, 1024), C::IDESC_PV,
+                 (first && kk == 0) ? 0u : 1u);
+      };
+      bool ok = mbar_wait(BAR(C::B_Q), 0, abort);
+      ok = ok && mbar_wait(BAR(C::B_FULL + 0), 0, abort);  // K_0 is sequence 0
+      tc_fence_after();
+      if (ok) {
+        issue_S(tmem + 0, qA, slot_addr(0));
+        mma_commit(BAR(C::B_S + 0));
+        if (hasB) {
+          issue_S(tmem + 128, qB, slot_addr(0));
+          mma_commit(BAR(C::B_S + 1));
+        }
+        mma_commit(BAR(C::B_EMPTY + 0));
+      }
+      for (int j = 0; ok && j < ntiles; ++j) {
+        const uint32_t vq = 2 * j + 1, kn = 2 * j + 2;
+        const bool more = j + 1 < ntiles;
+        ok = mbar_wait(BAR(C::B_FULL + vq % NS), (vq / NS) & 1, abort) &&
+             mbar_wait(BAR(C::B_P + 0), j & 1, abort);
+        if (!ok) break;
+        tc_fence_after();
+        issue_PV(tmem + 256, tmem + 0, slot_addr(vq), j == 0);
+        if (more) {
+          ok = mbar_wait(BAR(C::B_FULL + kn % NS), (kn / NS) & 1, abort);
+          if (!ok) break;
+          tc_fence_after();
+          issue_S(tmem + 0, qA, slot_addr(kn));
+          mma_commit(BAR(C::B_S + 0));
+        } else {
+          mma_commit(BAR(C::B_O + 0));
+        }
+        if (hasB) {
+          ok = mbar_wait(BAR(C::B_P + 1), j & 1, abort);
+          if (!ok) break;
+          tc_fence_after();
+          issue_PV(tmem + 256 + D, tmem + 128, slot_addr(vq), j == 0);
+          mma_commit(BAR(C::B_EMPTY + vq % NS));
+          if (more) {
+            issue_S(tmem + 128, qB, slot_addr(kn));
+            mma_commit(BAR(C::B_S + 1));
+            mma_commit(BAR(C::B_EMPTY + kn % NS));
+          } else {
+            mma_commit(BAR(C::B_O + 1));
+          }
+        } else {
+          mma_commit(BAR(C::B_EMPTY + vq % NS));
+          if (more) mma_commit(BAR(C::B_EMPTY + kn % NS));
+        }
+      }
+      if (ok && has_lin) {
+        // O += phi~(Q) [S_hi ; S_lo]: A = scaled phi(Q) in TMEM over the S
+        // columns, B = state rows (features) x D, MN-major, 128 rows a slot.
+        const uint32_t s0 = 2 * ntiles;
+        for (int i = 0; i < 2 * C::SPP && ok; ++i)
+          ok = mbar_wait(BAR(C::B_FULL + (s0 + i) % NS), ((s0 + i) / NS) & 1, abort);
+        for (int X = 0; X < (hasB ? 2 : 1) && ok; ++X) {
+          ok = mbar_wait(BAR(C::B_PHI + X), 0, abort);
+          if (!ok) break;
+          tc_fence_after();
+          for (int part = 0; part < 2; ++part) {
+#pragma unroll
+            for (int kk = 0; kk < (2 * D) / 16; ++kk) {
+              const uint32_t sa = slot_addr(s0 + part * C::SPP + kk / 8);
+              const uint32_t acc = PARTS ? ((part | kk) != 0 ? 1u : 0u) : 1u;
+              mma_ts(tmem + 256 + X * D, tmem + X * 128 + kk * 8,
+                     smem_desc_sw128(sa + (kk & 7) * 2048, C::BOX_BYTES, 1024), C::IDESC_PV, acc);
+            }
+          }
+          mma_commit(BAR(C::B_LIN + X));
+        }
+        if (ok)
+          for (int i = 0; i < 2 * C::SPP; ++i) mma_commit(BAR(C::B_EMPTY + (s0 + i) % NS));
+      }
+      // drain: all MMAs complete before TMEM is released
+      mma_commit(BAR(C::B_FIN));
+      drain_wait(BAR(C::B_FIN), 0);
+    }
+  }
+#undef BAR
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+// ============================================================================
+// Segment states: phi(K)^T V and sum phi(K)
+// ============================================================================
+template <int D>
+struct StCfg {
+  static constexpr int NBOX = D / 64;
+  static constexpr int BOX = 64 * 128;                // 64 token rows x 128 B
+  static constexpr int KV_BYTES = NBOX * BOX;         // 64 x D bf16
+  static constexpr int PHI_BYTES = 2 * NBOX * BOX;    // 64 x 2D bf16
+  static constexpr int STAGE = 2 * KV_BYTES + PHI_BYTES;
+  static constexpr int NST = (D == 128) ? 3 : 4;
+  static constexpr int HALVES = (2 * D) / 128;        // M = 128 feature blocks
+  static constexpr uint32_t TMEM_COLS = (HALVES * D <= 64) ? 64 : ((HALVES * D <= 128) ? 128 : 256);
+  static constexpr int OFF_BAR = NST * STAGE;
+  static constexpr int SMEM = OFF_BAR + 256 + 1024;
+  static constexpr int CH = D / 8;                    // 16-byte chunks per row
+  static constexpr int G = 128 / CH;                  // token groups over 128 threads
+  static constexpr int TPG = 64 / G;                  // tokens per thread per tile
+  static constexpr int B_KV = 0, B_PHI = NST, B_EMPTY = 2 * NST, B_ACC = 3 * NST, B_FIN = 3 * NST + 1;
+  // A = phi(K)^T (features x tokens, features contiguous: MN-major),
+  // B = V (tokens x D, D contiguous: MN-major).
+  static constexpr uint32_t IDESC = idesc_bf16_f32(128, D, 1, 1);
+  static_assert(SMEM <= 232448, "shared memory");
+  static_assert(G * CH == 128 && TPG * G == 64, "thread mapping");
+};
+
+template <int D>
+__global__ void __launch_bounds__(192, 1) phi_state_kernel(const __grid_constant__ StateParams p) {
+  using C = StCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int u = blockIdx.x;  // (bh * n_seg + s) * nsplit + piece
+  const int piece = u % p.sg.nsplit;
+  const int s = (u / p.sg.nsplit) % p.sg.n_seg;
+  const int bh = u / (p.sg.nsplit * p.sg.n_seg);
+  int a, b;
+  p.sg.piece(s, piece, a, b);
+  const int ntiles = cdiv(b - a, 64);
+  float* outS = p.part_S + static_cast<size_t>(u) * (2 * D) * D;
+  float* outz = p.part_z + static_cast<size_t>(u) * (2 * D);
+  if (ntiles == 0) {  // empty piece: its sums are zero
+    for (int i = threadIdx.x; i < 2 * D * D; i += blockDim.x) outS[i] = 0.f;
+    for (int i = threadIdx.x; i < 2 * D; i += blockDim.x) outz[i] = 0.f;
+    return;
+  }
+
+  uint8_t* barea = smem + C::OFF_BAR;
+  const uint32_t bar0 = smem_u32(barea);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(barea + 128);
+  volatile int* abort = reinterpret_cast<volatile int*>(barea + 132);
+#define BAR(i) (bar0 + 8u * static_cast<uint32_t>(i))
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < C::NST; ++i) {
+      mbar_init(BAR(C::B_KV + i), 1);
+      mbar_init(BAR(C::B_PHI + i), 128);
+      mbar_init(BAR(C::B_EMPTY + i), 1);
+    }
+    mbar_init(BAR(C::B_ACC), 1);
+    mbar_init(BAR(C::B_FIN), 1);
+    *abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 4 && lane == 0) {
+    prefetch_tmap(&p.tm_k);
+    prefetch_tmap(&p.tm_v);
+  }
+  if (warp == 5) {
+    tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp < 4) {
+    // ============ phi(K) into the MN-major A operand, sum phi(K) ============
+    // phi atom bx (< NBOX) = psi of dims 64bx..64bx+63, atom NBOX+bx = psi^2:
+    // byte-for-byte the same positions as the K box bx, so no re-layout.
+    const int tid = threadIdx.x;
+    const int c = tid % C::CH;
+    const int g = tid / C::CH;
+    const int bx = c >> 3, cc = c & 7;
+    float za[8], zb[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) za[e] = zb[e] = 0.f;
+    bool ok = true;
+    for (int i = 0; i < ntiles; ++i) {
+      const int st = i % C::NST;
+      ok = mbar_wait(BAR(C::B_KV + st), (i / C::NST) & 1, abort);
+      if (!ok) break;
+      const uint8_t* kt = smem + st * C::STAGE;
+      uint8_t* ph = smem + st * C::STAGE + 2 * C::KV_BYTES;
+#pragma unroll
+      for (int ii = 0; ii < C::TPG; ++ii) {
+        const int tok = g + ii * C::G;
+        const bool valid = a + 64 * i + tok < b;
+        const int off = tok * 128 + ((cc ^ (tok & 7)) << 4);
+        uint4 pa = make_uint4(0u, 0u, 0u, 0u), pb = pa;
+        if (valid) {
+          const uint4 raw = *reinterpret_cast<const uint4*>(kt + bx * C::BOX + off);
+          const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+          uint32_t va[4], vb[4];
+#pragma unroll
+          for (int h = 0; h < 4; ++h) {
+            const float s0 = psi1(bf16lo(w[h])), s1 = psi1(bf16hi(w[h]));
+            za[2 * h] += s0;
+            za[2 * h + 1] += s1;
+            zb[2 * h] += s0 * s0;
+            zb[2 * h + 1] += s1 * s1;
+            va[h] = pack_bf16(s0, s1);
+            vb[h] = pack_bf16(s0 * s0, s1 * s1);
+          }
+          pa = make_uint4(va[0], va[1], va[2], va[3]);
+          pb = make_uint4(vb[0], vb[1], vb[2], vb[3]);
+        }
+        *reinterpret_cast<uint4*>(ph + bx * C::BOX + off) = pa;
+        *reinterpret_cast<uint4*>(ph + (C::NBOX + bx) * C::BOX + off) = pb;
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(BAR(C::B_PHI + st));
+    }
+    // ---- epilogue: TMEM accumulators -> partial state rows ----
+    if (ok) ok = mbar_wait(BAR(C::B_ACC), 0, abort);
+    ok = __all_sync(kFull, ok);
+    tc_fence_after();
+    if (ok) {
+#pragma unroll
+      for (int h = 0; h < C::HALVES; ++h) {
+        const int e = 128 * h + 32 * warp + lane;
+#pragma unroll
+        for (int q = 0; q < D / 32; ++q) {
+          uint32_t v[32];
+          tmem_ld32(tmem + (static_cast<uint32_t>(32 * warp) << 16) + h * D + 32 * q, v);
+          tmem_ld_wait();
+          reg_fence(v);
+          float4* dst = reinterpret_cast<float4*>(outS + static_cast<size_t>(e) * D + 32 * q);
+#pragma unroll
+          for (int k4 = 0; k4 < 8; ++k4)
+            dst[k4] = make_float4(__uint_as_float(v[4 * k4]), __uint_as_float(v[4 * k4 + 1]),
+                                  __uint_as_float(v[4 * k4 + 2]), __uint_as_float(v[4 * k4 + 3]));
+        }
+      }
+      // sum phi(K) across the token groups (stage 0 is free: every MMA is done)
+      float* zred = reinterpret_cast<float*>(smem);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        zred[g * 2 * D + 8 * c + e] = za[e];
+        zred[g * 2 * D + D + 8 * c + e] = zb[e];
+      }
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      for (int f = tid; f < 2 * D; f += 128) {
+        float acc = 0.f;
+        for (int gg = 0; gg < C::G; ++gg) acc += zred[gg * 2 * D + f];
+        outz[f] = acc;
+      }
+    }
+  } else if (warp == 4) {
+    // =============================== TMA producer ============================
+    if (lane == 0) {
+      bool ok = true;
+      int i = 0;
+      for (; i < ntiles && ok; ++i) {
+        const int st = i % C::NST;
+        ok = mbar_wait(BAR(C::B_EMPTY + st), ((i / C::NST) & 1) ^ 1, abort);
+        if (!ok) break;
+        const uint32_t base = smem_u32(smem + st * C::STAGE);
+        mbar_arrive_expect_tx(BAR(C::B_KV + st), 2 * C::KV_BYTES);
+        for (int bb = 0; bb < C::NBOX; ++bb) {
+          tma_load_3d(base + bb * C::BOX, &p.tm_k, BAR(C::B_KV + st), 64 * bb, a + 64 * i, bh);
+          tma_load_3d(base + C::KV_BYTES + bb * C::BOX, &p.tm_v, BAR(C::B_KV + st), 64 * bb, a + 64 * i, bh);
+        }
+      }
+      for (int i2 = (i > C::NST ? i - C::NST : 0); i2 < i; ++i2)
+        drain_wait(BAR(C::B_KV + i2 % C::NST), (i2 / C::NST) & 1);
+    }
+  } else {
+    // =============================== MMA issuer ==============================
+    if (lane == 0) {
+      bool ok = true;
+      for (int i = 0; i < ntiles && ok; ++i) {
+        const int st = i % C::NST;
+        ok = mbar_wait(BAR(C::B_KV + st), (i / C::NST) & 1, abort) &&
+             mbar_wait(BAR(C::B_PHI + st), (i / C::NST) & 1, abort);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t vb = smem_u32(smem + st * C::STAGE + C::KV_BYTES);
+        const uint32_t pb = smem_u32(smem + st * C::STAGE + 2 * C::KV_BYTES);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {  // 16 tokens per MMA
+#pragma unroll
+          for (int h = 0; h < C::HALVES; ++h)
+            mma_ss(tmem + h * D, smem_desc_sw128(pb + 2 * h * C::BOX + kk * 2048, C::BOX, 1024),
+                   smem_desc_sw128(vb + kk * 2048, C::BOX, 1024), C::IDESC, (i > 0 || kk > 0) ? 1u : 0u);
+        }
+        mma_commit(BAR(C::B_EMPTY + st));
+      }
+      if (ok) mma_commit(BAR(C::B_ACC));
+      mma_commit(BAR(C::B_FIN));
+      drain_wait(BAR(C::B_FIN), 0);
+    }
+  }
+#undef BAR
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+// ============================================================================
+// Scan / accumulate / split (SIMT, memory-bound)
+// ============================================================================
+// One thread per state entry (bh, e, c) with c == D meaning z: walks the
+// chunks in order, writing the exclusive prefix, then adding segment t.
+__global__ void state_scan_kernel(const float* __restrict__ pS, const float* __restrict__ pz, int BH,
+                                  int n_seg, int nsplit, int nc, int D, __nv_bfloat16* hi,
+                                  __nv_bfloat16* lo, float* Sf, float* zt) {
+  const int W = D + 1;
+  const long long total = static_cast<long long>(BH) * 2 * D * W;
+  for (long long idx = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; idx < total;
+       idx += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const int c = static_cast<int>(idx % W);
+    const int e = static_cast<int>((idx / W) % (2 * D));
+    const int bh = static_cast<int>(idx / (static_cast<long long>(W) * 2 * D));
+    float acc = 0.f;
+    for (int t = 0; t < nc; ++t) {
+      const size_t so = ((static_cast<size_t>(bh) * nc + t) * 2 * D + e);
+      if (c == D) {
+        zt[so] = acc;
+      } else if (hi != nullptr) {
+        const __nv_bfloat16 h = __float2bfloat16_rn(acc);
+        hi[so * D + c] = h;
+        lo[so * D + c] = __float2bfloat16_rn(acc - __bfloat162float(h));
+      } else {
+        Sf[so * D + c] = acc;
+      }
+      if (t < n_seg) {
+        for (int pp = 0; pp < nsplit; ++pp) {
+          const size_t po = (static_cast<size_t>(bh) * n_seg + t) * nsplit + pp;
+          acc += (c == D) ? pz[po * 2 * D + e] : pS[(po * 2 * D + e) * D + c];
+        }
+      }
+    }
+  }
+}
+
+__global__ void state_accumulate_kernel(const float* __restrict__ pS, const float* __restrict__ pz, int BH,
+                                        int nsplit, int D, float* S, float* z) {
+  const int W = D + 1;
+  const long long total = static_cast<long long>(BH) * 2 * D * W;
+  for (long long idx = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; idx < total;
+       idx += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const int c = static_cast<int>(idx % W);
+    const int e = static_cast<int>((idx / W) % (2 * D));
+    const int bh = static_cast<int>(idx / (static_cast<long long>(W) * 2 * D));
+    float acc = 0.f;
+    for (int pp = 0; pp < nsplit; ++pp) {
+      const size_t po = static_cast<size_t>(bh) * nsplit + pp;
+      acc += (c == D) ? pz[po * 2 * D + e] : pS[(po * 2 * D + e) * D + c];
+    }
+    if (c == D)
+      z[static_cast<size_t>(bh) * 2 * D + e] += acc;
+    else
+      S[(static_cast<size_t>(bh) * 2 * D + e) * D + c] += acc;
+  }
+}
+
+__global__ void state_split_kernel(const float* __restrict__ S, long long n, __nv_bfloat16* hi,
+                                   __nv_bfloat16* lo) {
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const float x = S[i];
+    const __nv_bfloat16 h = __float2bfloat16_rn(x);
+    hi[i] = h;
+    lo[i] = __float2bfloat16_rn(x - __bfloat162float(h));
+  }
+}
+
+int grid_for(long long n, int threads) {
+  long long g = (n + threads - 1) / threads;
+  if (g > 148LL * 16) g = 148LL * 16;
+  return static_cast<int>(g < 1 ? 1 : g);
+}
+
+}  // namespace
+
+int attn_smem_bytes(int D) { return D == 128 ? AttnCfg<128>::SMEM : AttnCfg<64>::SMEM; }
+int state_smem_bytes(int D) { return D == 128 ? StCfg<128>::SMEM : StCfg<64>::SMEM; }
+
+template <int D, bool PARTS>
+static cudaError_t launch_attn_t(const AttnParams& p, int n_units, cudaStream_t s) {
+  auto* k = hybrid_chunk_attn_kernel<D, PARTS>;
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, AttnCfg<D>::SMEM);
+  if (e != cudaSuccess) return e;
+  k<<<n_units, 320, AttnCfg<D>::SMEM, s>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_attention(int D, bool parts, const AttnParams& p, int n_units, cudaStream_t s) {
+  if (n_units <= 0) return cudaSuccess;
+  if (D == 128) return parts ? launch_attn_t<128, true>(p, n_units, s) : launch_attn_t<128, false>(p, n_units, s);
+  return parts ? launch_attn_t<64, true>(p, n_units, s) : launch_attn_t<64, false>(p, n_units, s);
+}
+
+template <int D>
+static cudaError_t launch_state_t(const StateParams& p, int n_ctas, cudaStream_t s) {
+  auto* k = phi_state_kernel<D>;
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, StCfg<D>::SMEM);
+  if (e != cudaSuccess) return e;
+  k<<<n_ctas, 192, StCfg<D>::SMEM, s>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_chunk_state(int D, const StateParams& p, int n_ctas, cudaStream_t s) {
+  if (n_ctas <= 0) return cudaSuccess;
+  return D == 128 ? launch_state_t<128>(p, n_ctas, s) : launch_state_t<64>(p, n_ctas, s);
+}
+
+cudaError_t launch_state_scan(const float* part_S, const float* part_z, int BH, int n_seg, int nsplit,
+                              int n_chunks, int D, __nv_bfloat16* hi, __nv_bfloat16* lo, float* Sf,
+                              float* zt, cudaStream_t s) {
+  const long long n = static_cast<long long>(BH) * 2 * D * (D + 1);
+  state_scan_kernel<<<grid_for(n, 256), 256, 0, s>>>(part_S, part_z, BH, n_seg, nsplit, n_chunks, D, hi, lo,
+                                                      Sf, zt);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_state_accumulate(const float* part_S, const float* part_z, int BH, int nsplit, int D,
+                                    float* state_S, float* state_z, cudaStream_t s) {
+  const long long n = static_cast<long long>(BH) * 2 * D * (D + 1);
+  state_accumulate_kernel<<<grid_for(n, 256), 256, 0, s>>>(part_S, part_z, BH, nsplit, D, state_S, state_z);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_state_split(const float* S, long long n, __nv_bfloat16* hi, __nv_bfloat16* lo,
+                               cudaStream_t s) {
+  state_split_kernel<<<grid_for(n, 256), 256, 0, s>>>(S, n, hi, lo);
+  return cudaGetLastError();
+}
+
+}  // namespace rehyat
+
+namespace rehyat {
+cudaError_t read_and_clear_device_error(unsigned int* v) {
+  cudaError_t e = cudaMemcpyFromSymbol(v, g_device_error, sizeof(unsigned int));
+  if (e != cudaSuccess) return e;
+  const unsigned int zero = 0;
+  return cudaMemcpyToSymbol(g_device_error, &zero, sizeof(unsigned int));
+}
+}  // namespace rehyat

@@ -10,9 +10,15 @@ be regenerated alone for sampled-row checks):
   stream(seed, which, b, h) = default_rng(SeedSequence([seed, which, b, h]))
   which: 0 = q, 1 = k, 2 = v;  x = scale * standard_normal((N, d)) in float64
   rms_qk: q, k -> x / sqrt(mean(x**2, axis=-1) + 1e-6)
+  post:   optional per-tensor factors applied after the RMS step (to make the
+          softmax branch dominate, or the linear one, in targeted tests)
   storage: float32, then bfloat16 by round-to-nearest-even (torch's cast).
+Heads are generated in parallel threads; the result does not depend on that.
 """
 from __future__ import annotations
+
+import os
+from concurrent.futures import ThreadPoolExecutor
 
 import numpy as np
 import torch
@@ -21,13 +27,13 @@ WHICH = {"q": 0, "k": 1, "v": 2}
 
 
 def head_array(seed: int, which: str, b: int, h: int, N: int, d: int,
-               scale: float = 1.0, rms_qk: bool = False) -> np.ndarray:
+               scale: float = 1.0, rms_qk: bool = False, post: float = 1.0) -> np.ndarray:
     """float64 [N, d] draw for one (tensor, batch, head)."""
     rng = np.random.default_rng(np.random.SeedSequence([seed, WHICH[which], b, h]))
     x = rng.standard_normal((N, d)) * scale
     if rms_qk and which in ("q", "k"):
         x = x / np.sqrt(np.mean(x * x, axis=-1, keepdims=True) + 1e-6)
-    return x
+    return x * post if post != 1.0 else x
 
 
 def _store(x64: np.ndarray, dtype: str) -> torch.Tensor:
@@ -40,20 +46,23 @@ def _store(x64: np.ndarray, dtype: str) -> torch.Tensor:
 
 
 def make_qkv(B: int, H: int, N: int, d: int, seed: int, dtype: str = "bf16",
-             scale: float = 1.0, rms_qk: bool = False, scales=None):
+             scale: float = 1.0, rms_qk: bool = False, post=(1.0, 1.0, 1.0), pin: bool = False):
     """Host tensors q, k, v of shape [B, H, N, d] in the storage dtype.
 
-    scales: optional (sq, sk, sv) overriding ``scale`` per tensor (used to
-    push the softmax branch to dominate, or the linear branch).
+    scale multiplies the N(0,1) draw; post = (sq, sk, sv) multiplies each
+    tensor after the optional RMS normalisation.  pin: page-locked memory.
     """
-    sc = scales if scales is not None else (scale, scale, scale)
-    out = []
-    for which, s in zip(("q", "k", "v"), sc):
-        t = torch.empty((B, H, N, d), dtype=torch.bfloat16 if dtype == "bf16" else torch.float32)
-        for b in range(B):
-            for h in range(H):
-                t[b, h] = _store(head_array(seed, which, b, h, N, d, s, rms_qk), dtype)
-        out.append(t)
+    tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
+    out = [torch.empty((B, H, N, d), dtype=tdt, pin_memory=pin) for _ in range(3)]
+    jobs = [(i, which, b, h) for i, which in enumerate(("q", "k", "v")) for b in range(B) for h in range(H)]
+
+    def fill(job):
+        i, which, b, h = job
+        out[i][b, h] = _store(head_array(seed, which, b, h, N, d, scale, rms_qk, post[i]), dtype)
+
+    workers = max(1, min(len(jobs), len(os.sched_getaffinity(0))))
+    with ThreadPoolExecutor(workers) as ex:
+        list(ex.map(fill, jobs))
     return tuple(out)
 
 

@@ -1,0 +1,122 @@
+"""C ABI checks that need no GPU: the library loads, exports every entry point
+declared in include/rehyat.h, and validates arguments on the host (returning a
+status without touching CUDA)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from linear_attention_video_chunk_b200 import build as rbuild
+from linear_attention_video_chunk_b200 import rehyat as R
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "rehyat.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    rbuild.build()
+    return R.lib()
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(rehyat_\w+)\s*\(", src)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for n in ("rehyat_forward", "rehyat_forward_f32", "rehyat_step", "rehyat_step_f32",
+              "rehyat_forward_parts", "rehyat_status_string"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    missing = [n for n in declared_functions() if not hasattr(lib, n)]
+    assert not missing, missing
+
+
+def test_binding_covers_every_symbol():
+    assert set(declared_functions()) <= set(R._SIGS)
+
+
+def test_only_c_abi_symbols_are_exported(lib):
+    out = os.popen(f"nm -D --defined-only {R.LIB_PATH}").read()
+    syms = [l.split()[-1] for l in out.splitlines() if " T " in l]
+    assert syms and all(s.startswith("rehyat_") for s in syms), syms
+
+
+def test_status_strings(lib):
+    for st in range(6):
+        assert R.status_string(st).startswith("REHYAT_")
+    assert "UNKNOWN" in R.status_string(99)
+
+
+def _fwd(lib, q=16, k=16, v=16, out=16, B=1, H=1, F=4, S=8, d=64, Tc=2, To=1):
+    return lib.rehyat_forward(q, k, v, B, H, F, S, d, Tc, To, out, None)
+
+
+def test_forward_validation(lib):
+    assert _fwd(lib, q=0) == R.EINVAL                     # null pointer
+    assert _fwd(lib, k=8) == R.EINVAL                     # 16-byte misaligned
+    assert _fwd(lib, d=96) == R.EUNSUPPORTED
+    assert _fwd(lib, d=0) == R.EINVAL
+    assert _fwd(lib, F=0) == R.EINVAL
+    assert _fwd(lib, S=0) == R.EINVAL
+    assert _fwd(lib, Tc=0) == R.EINVAL
+    assert _fwd(lib, To=-1) == R.EINVAL
+    assert _fwd(lib, B=-1) == R.EINVAL
+    assert _fwd(lib, F=1 << 20, S=1 << 12) == R.EINVAL   # N overflows int
+    assert lib.rehyat_forward_f32(0, 16, 16, 1, 1, 4, 8, 64, 2, 1, 16, None) == R.EINVAL
+    assert lib.rehyat_forward_parts(16, 16, 16, 1, 1, 4, 8, 64, 2, 1, 0, 16, 16, 16, 16, None) == R.EINVAL
+
+
+def test_step_validation(lib):
+    st = lambda **kw: lib.rehyat_step(*(kw.get(n, 16) for n in ("q", "k", "v", "S", "z", "o")),
+                                      1, 1, 8, kw.get("d", 64), kw.get("qf", 2), kw.get("cf", 1),
+                                      kw.get("ef", 1), None)
+    assert st(S=0) == R.EINVAL
+    assert st(z=4) == R.EINVAL
+    assert st(ef=4) == R.EINVAL        # evict beyond the window
+    assert st(qf=0) == R.EINVAL
+    assert st(cf=-1) == R.EINVAL
+    assert st(d=32) == R.EUNSUPPORTED
+
+
+def test_workspace_sizes(lib):
+    a = R.workspace_bytes(1, 12, 21, 1560, 128, 3, 1)
+    b = R.workspace_bytes(1, 12, 41, 1560, 128, 3, 1)
+    assert 0 < a < b and a % 256 == 0
+    # the states of 7 chunks (bf16 hi + lo + fp32 z) are part of it
+    assert a >= 12 * 7 * 256 * 128 * 2 * 2
+    assert R.workspace_bytes(1, 1, 4, 8, 64, 4, 0) >= 256          # one chunk: no segments
+    assert R.step_workspace_bytes(1, 12, 1560, 128, 3, 1, 3) > 0
+    n = ctypes.c_size_t(0)
+    assert lib.rehyat_forward_workspace_bytes(1, 1, 4, 8, 64, 2, 1, None) == R.EINVAL
+    assert lib.rehyat_forward_workspace_bytes(1, 1, 4, 8, 100, 2, 1, ctypes.byref(n)) == R.EUNSUPPORTED
+
+
+def test_ws_variants_check_workspace(lib):
+    # workspace too small -> ENOMEM before any launch; misaligned -> EINVAL
+    assert lib.rehyat_forward_ws(16, 16, 16, 1, 1, 4, 8, 64, 2, 1, 16, 256, 1, None) == R.ENOMEM
+    assert lib.rehyat_forward_ws(16, 16, 16, 1, 1, 4, 8, 64, 2, 1, 16, 272, 1 << 30, None) == R.EINVAL
+
+
+def test_phi_validation(lib):
+    assert lib.rehyat_phi(0, 0, 16, 0, 4, 64, None) == R.EINVAL
+    assert lib.rehyat_phi(16, 3, 16, 0, 4, 64, None) == R.EINVAL
+    assert lib.rehyat_phi(16, 0, 16, 0, 0, 64, None) == R.EINVAL
+
+
+def test_step_frames_cover_the_video():
+    """Host logic of the streaming driver: windows and evictions tile [0, F)."""
+    for F, Tc, To in [(21, 3, 1), (81, 3, 1), (7, 2, 3), (10, 4, 0), (5, 7, 2)]:
+        folded = 0
+        t = 0
+        while t * min(Tc, F) < F:
+            f0, w, cf, qf, ef = R.step_frames(t, F, Tc, To)
+            assert w == folded and cf == f0 - w and qf >= 1
+            folded += ef
+            t += 1
+        assert folded <= F

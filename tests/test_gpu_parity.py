@@ -1,0 +1,271 @@
+"""GPU parity: the CUDA library (through its C ABI) against the fp64 oracle.
+
+Tolerances (the benchmark spec): fp32 paths max relative L2 error <= 1e-5; bf16 paths
+relative L2 <= 1e-2 and max |error| <= 3e-2 * RMS(reference).  Relative L2 is
+taken per (b, h) over the compared rows and the maximum over (b, h) is
+checked.  Inputs come from the shared seeded generator; the oracle sees the
+exact stored values (bf16 or fp32) widened to fp64.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle.rehyat_oracle as orc
+from linear_attention_video_chunk_b200 import inputs
+from linear_attention_video_chunk_b200 import rehyat as R
+
+pytestmark = pytest.mark.gpu
+
+F32_TOL = 1e-5
+BF16_L2 = 1e-2
+BF16_MAX = 3e-2
+
+
+def rel_l2(y, ref):
+    y = np.asarray(y, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    num = np.sqrt(((y - ref) ** 2).sum(axis=(-2, -1)))
+    den = np.sqrt((ref ** 2).sum(axis=(-2, -1)))
+    return float((num / den).max())
+
+
+def max_over_rms(y, ref):
+    y = np.asarray(y, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    return float(np.abs(y - ref).max() / np.sqrt((ref ** 2).mean()))
+
+
+def assert_bf16_close(y, ref, what=""):
+    e2, em = rel_l2(y, ref), max_over_rms(y, ref)
+    assert e2 <= BF16_L2 and em <= BF16_MAX, f"{what}: rel L2 {e2:.3e}, max/RMS {em:.3e}"
+    return e2, em
+
+
+def np64(t):
+    return t.detach().float().cpu().double().numpy()
+
+
+def sample_rows(F, S_tok, Tc, edge=64, n_rand=256, seed=7):
+    """First and last `edge` rows of every chunk plus random rows."""
+    N = F * S_tok
+    Np = min(Tc, F) * S_tok
+    rows = set()
+    for q0 in range(0, N, Np):
+        q1 = min(q0 + Np, N)
+        rows.update(range(q0, min(q0 + edge, q1)))
+        rows.update(range(max(q1 - edge, q0), q1))
+    rows.update(np.random.default_rng(seed).integers(0, N, n_rand).tolist())
+    return np.array(sorted(rows))
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    R.lib()
+    yield
+    assert R.device_status() == R.OK, "a device-side wait timed out"
+
+
+# --------------------------------------------------------------------------- #
+# fp32 path                                                                    #
+# --------------------------------------------------------------------------- #
+F32_CASES = [
+    # B, H, d, F, S_tok, Tc, To, seed   (first: the tiny fp32 oracle-check config)
+    (1, 2, 64, 4, 64, 2, 1, 0),
+    (2, 1, 128, 5, 24, 2, 1, 10),
+    (1, 2, 64, 7, 9, 3, 4, 11),      # overlap longer than a chunk, ragged
+    (1, 1, 128, 4, 16, 6, 1, 12),    # one chunk (full softmax)
+    (1, 3, 64, 6, 10, 1, 0, 13),     # no overlap, one-frame chunks
+    (1, 1, 64, 1, 33, 2, 1, 14),     # a single frame
+]
+
+
+@pytest.mark.parametrize("B,H,d,F,S,Tc,To,seed", F32_CASES)
+def test_forward_f32_matches_oracle(B, H, d, F, S, Tc, To, seed):
+    q, k, v = inputs.make_qkv(B, H, F * S, d, seed, dtype="f32", scale=0.5)
+    y = R.forward_f32(q.cuda(), k.cuda(), v.cuda(), F, S, Tc, To)
+    ref = orc.oracle_forward(q, k, v, F, S, Tc, To)
+    e = rel_l2(np64(y), ref)
+    assert e <= F32_TOL, e
+
+
+def test_step_f32_streamed_matches_oracle():
+    B, H, d, F, S, Tc, To = 1, 2, 64, 7, 16, 2, 1
+    q, k, v = inputs.make_qkv(B, H, F * S, d, 20, dtype="f32", scale=0.5)
+    qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+    Sst = torch.zeros(B, H, 2 * d, d, device="cuda")
+    zst = torch.zeros(B, H, 2 * d, device="cuda")
+    outs = []
+    t = 0
+    while t * Tc < F:
+        f0, w, cf, qf, ef = R.step_frames(t, F, Tc, To)
+        outs.append(R.step_f32(qd[:, :, f0 * S:(f0 + qf) * S].contiguous(), kd[:, :, w * S:(f0 + qf) * S].contiguous(),
+                               vd[:, :, w * S:(f0 + qf) * S].contiguous(), Sst, zst, S, qf, cf, ef))
+        t += 1
+    y = torch.cat(outs, dim=2)
+    ref = orc.oracle_forward(q, k, v, F, S, Tc, To)
+    assert rel_l2(np64(y), ref) <= F32_TOL
+
+
+# --------------------------------------------------------------------------- #
+# bf16 tensor-core path, full oracle                                           #
+# --------------------------------------------------------------------------- #
+BF16_CASES = [
+    # B, H, d, F, S_tok, Tc, To, seed
+    (1, 2, 128, 5, 200, 2, 1, 30),    # ragged windows and last chunk
+    (1, 2, 64, 5, 200, 2, 1, 31),     # d = 64
+    (2, 1, 128, 7, 96, 3, 1, 32),     # B = 2, tiles aligned to 128
+    (1, 1, 128, 6, 70, 2, 3, 33),     # overlap longer than a chunk
+    (1, 2, 128, 4, 150, 1, 0, 34),    # no overlap
+    (1, 1, 128, 3, 180, 4, 1, 35),    # one chunk: full softmax over 540 keys
+    (1, 1, 128, 1, 77, 3, 1, 36),     # one short frame (single 77-row tile)
+    (1, 1, 128, 9, 40, 2, 1, 37),     # short frames, many chunks
+    (1, 1, 64, 3, 300, 1, 1, 38),     # 300-row chunks (a lone 44-row tile B)
+]
+
+
+@pytest.mark.parametrize("B,H,d,F,S,Tc,To,seed", BF16_CASES)
+def test_forward_bf16_matches_oracle(B, H, d, F, S, Tc, To, seed):
+    q, k, v = inputs.make_qkv(B, H, F * S, d, seed, rms_qk=True)
+    y = R.forward(q.cuda(), k.cuda(), v.cuda(), F, S, Tc, To)
+    ref = orc.oracle_forward(q, k, v, F, S, Tc, To)
+    assert_bf16_close(np64(y), ref)
+
+
+@pytest.mark.parametrize("post", [(8.0, 1.0, 1.0), (3.0, 1.0, 1.0), (0.25, 0.25, 1.0)])
+def test_forward_bf16_softmax_and_linear_balance(post):
+    """Scaled queries move the balance between the branches: q x 8 makes the
+    softmax window dominate every chunk, q x 3 mixes both, q,k x 0.25 makes
+    scores flat so the linear term dominates."""
+    B, H, d, F, S, Tc, To = 1, 2, 128, 5, 160, 2, 1
+    q, k, v = inputs.make_qkv(B, H, F * S, d, 40, rms_qk=True, post=post)
+    y = R.forward(q.cuda(), k.cuda(), v.cuda(), F, S, Tc, To)
+    assert_bf16_close(np64(y), orc.oracle_forward(q, k, v, F, S, Tc, To), str(post))
+
+
+def test_forward_parts_match_oracle_parts():
+    """Each branch separately (the linear term dominates the output, so the
+    final y alone cannot pin the softmax branch of later chunks)."""
+    B, H, d, F, S, Tc, To = 1, 2, 128, 5, 200, 2, 1
+    q, k, v = inputs.make_qkv(B, H, F * S, d, 41, rms_qk=True)
+    aS, nS, aL, nL, M = (np64(x) for x in R.forward_parts(q.cuda(), k.cuda(), v.cuda(), F, S, Tc, To))
+    oS, onS, oL, onL = orc.oracle_parts(q, k, v, F, S, Tc, To)
+    assert_bf16_close(aS / nS[..., None], oS / onS[..., None], "softmax branch")
+    lin = onL > 0
+    assert (nL[~lin] == 0).all() and (aL[~lin] == 0).all()
+    rows = lin[0, 0]
+    assert_bf16_close((aL / nL[..., None])[:, :, rows], (oL / onL[..., None])[:, :, rows], "linear branch")
+    mix = (nS / nL)[lin]
+    omix = (onS / onL)[lin]
+    assert np.abs(mix / omix - 1).max() < 2e-3
+    y = (aS + aL) / (nS + nL)[..., None]
+    assert_bf16_close(y, orc.oracle_forward(q, k, v, F, S, Tc, To), "recombined")
+    assert np.isfinite(M).all() and (M[lin] >= 0).all()
+
+
+@pytest.mark.parametrize("B,H,d,F,S,Tc,To", [(1, 2, 128, 7, 100, 2, 1), (1, 1, 64, 6, 90, 2, 3),
+                                            (1, 1, 128, 5, 64, 1, 0)])
+def test_chunk_states_match_oracle(B, H, d, F, S, Tc, To):
+    q, k, v = inputs.make_qkv(B, H, F * S, d, 50, rms_qk=True)
+    Sg, zg = R.chunk_states(k.cuda(), v.cuda(), F, S, Tc, To)
+    So, zo = orc.oracle_chunk_states(k, v, F, S, Tc, To)
+    Sg, zg = np64(Sg), np64(zg)
+    assert (Sg[:, :, 0] == 0).all() and (zg[:, :, 0] == 0).all()
+    for t in range(1, So.shape[2]):
+        if np.abs(zo[:, :, t]).max() == 0:
+            continue
+        eS = np.linalg.norm(Sg[:, :, t] - So[:, :, t]) / np.linalg.norm(So[:, :, t])
+        ez = np.abs(zg[:, :, t] - zo[:, :, t]).max() / np.abs(zo[:, :, t]).max()
+        assert eS < 1e-2 and ez < 1e-3, (t, eS, ez)
+
+
+def test_forward_capi_and_stages_agree_bitwise():
+    B, H, d, F, S, Tc, To = 1, 2, 128, 6, 130, 3, 1
+    q, k, v = (x.cuda() for x in inputs.make_qkv(B, H, F * S, d, 60, rms_qk=True))
+    a = R.forward(q, k, v, F, S, Tc, To)
+    b = R.forward_capi(q, k, v, F, S, Tc, To)
+    ws = R.alloc_workspace(R.workspace_bytes(B, H, F, S, d, Tc, To), q.device)
+    c = torch.empty_like(q)
+    R.forward_states(k, v, F, S, Tc, To, ws)
+    R.forward_attention(q, k, v, F, S, Tc, To, c, ws)
+    d2 = R.forward(q, k, v, F, S, Tc, To)
+    assert torch.equal(a, b) and torch.equal(a, c) and torch.equal(a, d2)
+
+
+def test_step_bf16_streamed_matches_forward_and_oracle():
+    B, H, d, F, S, Tc, To = 1, 2, 128, 8, 120, 3, 1
+    q, k, v = inputs.make_qkv(B, H, F * S, d, 70, rms_qk=True)
+    qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+    Sst = torch.zeros(B, H, 2 * d, d, device="cuda")
+    zst = torch.zeros(B, H, 2 * d, device="cuda")
+    outs = []
+    t = 0
+    while t * Tc < F:
+        f0, w, cf, qf, ef = R.step_frames(t, F, Tc, To)
+        outs.append(R.step(qd[:, :, f0 * S:(f0 + qf) * S].contiguous(), kd[:, :, w * S:(f0 + qf) * S].contiguous(),
+                           vd[:, :, w * S:(f0 + qf) * S].contiguous(), Sst, zst, S, qf, cf, ef, capi=(t % 2 == 1)))
+        t += 1
+    y = np64(torch.cat(outs, dim=2))
+    ref = orc.oracle_forward(q, k, v, F, S, Tc, To)
+    assert_bf16_close(y, ref, "step vs oracle")
+    yf = np64(R.forward(qd, kd, vd, F, S, Tc, To))
+    assert rel_l2(y, yf) <= 5e-3
+    # the carried state equals the sum over every folded key
+    So, zo = orc.oracle_chunk_states(k, v, F, S, Tc, To)
+    # after the last step the state covers [0, w_last + evicted) = all keys before
+    # the end of the video minus nothing left in the last window's tail
+    f0, w, cf, qf, ef = R.step_frames(t - 1, F, Tc, To)
+    n_fold = (w + ef) * S
+    PK = orc.phi(k[:, :, :n_fold].double().numpy())
+    S_ref = np.einsum("bhje,bhjc->bhec", PK, v[:, :, :n_fold].double().numpy())
+    assert np.linalg.norm(np64(Sst) - S_ref) / np.linalg.norm(S_ref) < 1e-2
+    assert np.abs(np64(zst) - PK.sum(2)).max() / np.abs(PK.sum(2)).max() < 1e-3
+
+
+def test_step_from_nonzero_state_matches_oracle_step():
+    B, H, d, S, qf, cf, ef = 1, 2, 128, 96, 2, 1, 2
+    q, _, _ = inputs.make_qkv(B, H, qf * S, d, 80, rms_qk=True)
+    _, k, v = inputs.make_qkv(B, H, (cf + qf) * S, d, 81, rms_qk=True)
+    S0, z0 = inputs.make_state(B, H, d, 82, scale=30.0)
+    Sd, zd = S0.cuda(), z0.cuda()
+    y = R.step(q.cuda(), k.cuda(), v.cuda(), Sd, zd, S, qf, cf, ef)
+    oy, oS, oz = orc.oracle_step(q, k, v, S0, z0, S, ef)
+    assert_bf16_close(np64(y), oy)
+    assert np.linalg.norm(np64(Sd) - oS) / np.linalg.norm(oS) < 1e-2
+    assert np.abs(np64(zd) - oz).max() / np.abs(oz).max() < 1e-3
+
+
+def test_deterministic_bitwise():
+    B, H, d, F, S, Tc, To = 1, 3, 128, 7, 110, 3, 1
+    q, k, v = (x.cuda() for x in inputs.make_qkv(B, H, F * S, d, 90, rms_qk=True))
+    a = R.forward(q, k, v, F, S, Tc, To)
+    for _ in range(3):
+        assert torch.equal(a, R.forward(q, k, v, F, S, Tc, To))
+
+
+@pytest.mark.parametrize("xd,yd", [(torch.float32, torch.float32), (torch.bfloat16, torch.float32),
+                                   (torch.bfloat16, torch.bfloat16)])
+def test_phi_kernel(xd, yd):
+    x = (torch.randn(1000, 128, generator=torch.Generator().manual_seed(5)) * 3).to(xd)
+    y = R.phi(x.cuda(), yd).cpu()
+    ref = orc.phi(x.double().numpy())
+    if yd == torch.float32:
+        np.testing.assert_allclose(y.double().numpy(), ref, rtol=2e-6, atol=1e-30)
+    else:
+        np.testing.assert_allclose(y.double().numpy(), ref, rtol=2 ** -8, atol=1e-30)
+
+
+# --------------------------------------------------------------------------- #
+# full-size configurations, sampled rows                                       #
+# --------------------------------------------------------------------------- #
+def test_wan13b_480p_sampled_rows():
+    """B=1, H=12, d=128, F=21 x 1560 tokens (32,760), T_c=3, T_o=1: the
+    benchmarked launch (rehyat_forward_ws), checked on the first/last 64 rows
+    of every chunk plus 256 random rows, every head."""
+    B, H, d, F, S, Tc, To = 1, 12, 128, 21, 1560, 3, 1
+    q, k, v = inputs.make_qkv(B, H, F * S, d, 1, rms_qk=True)
+    y = R.forward(q.cuda(), k.cuda(), v.cuda(), F, S, Tc, To).cpu()
+    rows = sample_rows(F, S, Tc)
+    ref = orc.oracle_forward(q, k, v, F, S, Tc, To, rows=rows)
+    assert_bf16_close(np64(y[:, :, rows]), ref)
