@@ -68,6 +68,27 @@ def work(c):
                 state_bytes=state_bytes, tokens=B * N)
 
 
+KERNEL_SOURCES = ("tc_kernels.cu", "ptx.cuh", "kernels.cuh", "geom.cuh")
+TRAFFIC_PROFILE = os.path.join(ROOT, "profiles", "hybrid_chunk_attn_h6_full.md")
+
+
+def attn_traffic(c):
+    """DRAM bytes per full launch from the committed ncu summary, or None if
+    the kernel sources changed since it was captured (or the workload differs)."""
+    import hashlib
+    try:
+        csrc = os.path.join(ROOT, "linear_attention_video_chunk_b200", "csrc")
+        h = hashlib.sha256(b"".join(open(os.path.join(csrc, f), "rb").read() for f in KERNEL_SOURCES)).hexdigest()
+        txt = open(TRAFFIC_PROFILE).read()
+        sha = txt.split("- source_sha256:")[1].split()[0]
+        nbytes = int(txt.split("- dram_bytes_per_full_launch:")[1].split()[0])
+    except Exception:
+        return None
+    if sha != h or (c["B"], c["H"], c["F"], c["S_tok"]) != (1, 12, 21, 1560):
+        return None
+    return nbytes
+
+
 def peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -85,14 +106,19 @@ class ClockSampler:
     REASONS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown",
                0x4: "sw_power_cap", 0x80: "hw_power_brake_slowdown", 0x1: "gpu_idle"}
 
-    def __init__(self, index):
+    def __init__(self, dev):
         self.samples, self.reasons, self.max_mhz = [], set(), None
         self._stop = threading.Event()
         try:
             import pynvml
+            import torch
             pynvml.nvmlInit()
             self.nv = pynvml
-            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            try:  # NVML enumerates every GPU; match the CUDA device by UUID
+                uuid = str(torch.cuda.get_device_properties(dev).uuid)
+                self.h = pynvml.nvmlDeviceGetHandleByUUID(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+            except Exception:
+                self.h = pynvml.nvmlDeviceGetHandleByIndex(dev.index or 0)
             self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
         except Exception:
             self.nv = None
@@ -204,7 +230,7 @@ def run_forward_bench(args, c, rank, world, dev):
     K = args.steps
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with ClockSampler(dev.index if dev.index is not None else 0) as clk:
+    with ClockSampler(dev) as clk:
         start.record()
         for i in range(K):
             step(*ev[i])
@@ -218,6 +244,9 @@ def run_forward_bench(args, c, rank, world, dev):
 
     # end to end through the public API: pinned host inputs -> device ->
     # forward -> result back to pinned host memory, every step
+    if args.no_e2e:
+        return dict(ms_step=ms_step, attn_ms=attn_ms, state_ms=state_ms, e2e_ms=float("nan"), clocks=clk.summary(),
+                    h2d=0, d2h=0, q=q, k=k, v=v, launches=3 * K)
     out_h = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
     Ke = max(3, min(K, 20))
     for _ in range(2):
@@ -258,6 +287,9 @@ def run_ours(args):
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     c = dict(CONFIGS[args.config])
+    if args.heads:
+        c["H"] = args.heads
+        c["workload"] += f" (H overridden to {args.heads})"
     if args.config == "recurrent":
         res = run_recurrent_bench(args, c, rank, world, dev)
     else:
@@ -280,7 +312,8 @@ def run_ours(args):
         line["roofline"] = {
             "kernel": "hybrid_chunk_attn_kernel", "bound": "tensor", "achieved": achieved, "peak": bf16_peak,
             "unit": "TFLOP/s", "frac": achieved / bf16_peak, "peak_source": f"{src} bf16 dense (burst)",
-            "frac_of_sustained": achieved / bf16_sus if bf16_sus else None, "traffic": None,
+            "frac_of_sustained": achieved / bf16_sus if bf16_sus else None, "traffic": attn_traffic(c),
+            "algorithmic_bytes": w["attn_bytes"],
             "kernel_ms": res["attn_ms"], "flops_per_launch": w["attn_flops"],
             "states_stage_ms": res["state_ms"],
             "path_frac": (w["attn_flops"] + w["state_flops"]) / (res["ms_step"] / 1e3) / 1e12 / bf16_peak,
@@ -289,7 +322,7 @@ def run_ours(args):
                    "d2h_bytes_per_step": res["d2h"], "ms_per_step": res["e2e_ms"]}
     line["clocks"] = res["clocks"]
     line["gpu_launches"] = res["launches"]
-    if rank == 0 and world == 1 and not args.no_cpu_baseline and args.config == "wan13b":
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and args.config == "wan13b" and not args.heads:
         rate, n, dt = oracle_sample_rate(c, res["q"], res["k"], res["v"], args.cpu_budget)
         line["cpu_baseline"] = {"value": rate, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
                                 "sample": f"fp64 explicit-mask oracle on {n} random query rows x all {c['H']} "
@@ -333,7 +366,7 @@ def run_recurrent_bench(args, c, rank, world, dev):
     torch.cuda.synchronize()
     K = max(1, args.steps // 10)
     s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with ClockSampler(dev.index or 0) as clk:
+    with ClockSampler(dev) as clk:
         s0.record()
         for _ in range(K):
             video()
@@ -437,6 +470,8 @@ def main():
     ap.add_argument("--config", choices=tuple(CONFIGS), default="wan13b")
     ap.add_argument("--sweep", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end leg (profiling runs)")
+    ap.add_argument("--heads", type=int, default=0, help="override H (smaller profiling cases)")
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work for cpu_baseline")
     args = ap.parse_args()
     if args.warmup < 3:

@@ -183,17 +183,19 @@ __global__ void __launch_bounds__(320, 1) hybrid_chunk_attn_kernel(const __grid_
         reg_fence(s[2]);
         reg_fence(s[3]);
         const int valid = win - j * 128;  // keys of this tile inside the window
-        float mx = -INFINITY;
+        if (valid < 128) {                 // only the window's last tile is partial
 #pragma unroll
-        for (int a = 0; a < 4; ++a) {
+          for (int a = 0; a < 4; ++a)
 #pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            float x = __uint_as_float(s[a][c]) * p.scale_log2;
-            x = (a * 32 + c < valid) ? x : -INFINITY;
-            s[a][c] = __float_as_uint(x);
-            mx = fmaxf(mx, x);
-          }
+            for (int c = 0; c < 32; ++c)
+              if (a * 32 + c >= valid) s[a][c] = __float_as_uint(-INFINITY);
         }
+        float mraw = -INFINITY;  // scale > 0, so the max is taken on raw scores
+#pragma unroll
+        for (int a = 0; a < 4; ++a)
+#pragma unroll
+          for (int c = 0; c < 32; ++c) mraw = fmaxf(mraw, __uint_as_float(s[a][c]));
+        const float mx = mraw * p.scale_log2;
         // Lazy rescaling: move the shift only when the row maximum exceeds
         // it by more than 2^8, so P <= 256 and fp32 sums stay exact enough.
         const bool need = mx > m_used + 8.f;
@@ -201,16 +203,19 @@ __global__ void __launch_bounds__(320, 1) hybrid_chunk_attn_kernel(const __grid_
         const float mnew = need ? mx : m_used;
         const float alpha = need ? ex2(m_used - mnew) : 1.f;
         m_used = mnew;
+        const float neg_m = -m_used;
         float rs = 0.f;
         uint32_t pk[2][32];
 #pragma unroll
         for (int a = 0; a < 4; ++a) {
 #pragma unroll
           for (int c = 0; c < 16; ++c) {
-            const float p0 = ex2(__uint_as_float(s[a][2 * c]) - m_used);
-            const float p1 = ex2(__uint_as_float(s[a][2 * c + 1]) - m_used);
-            rs += p0 + p1;
-            pk[a >> 1][(a & 1) * 16 + c] = pack_bf16(p0, p1);
+            const float p0 = ex2(fmaf(__uint_as_float(s[a][2 * c]), p.scale_log2, neg_m));
+            const float p1 = ex2(fmaf(__uint_as_float(s[a][2 * c + 1]), p.scale_log2, neg_m));
+            const uint32_t u = pack_bf16(p0, p1);
+            // the denominator sums exactly the bf16 weights the P.V MMA uses
+            rs += bf16lo(u) + bf16hi(u);
+            pk[a >> 1][(a & 1) * 16 + c] = u;
           }
         }
         l = l * alpha + rs;
@@ -263,9 +268,9 @@ __global__ void __launch_bounds__(320, 1) hybrid_chunk_attn_kernel(const __grid_
       }
 
       // ---- linear term: phi(q) S_t and phi(q) z_t (§3.1 cached sums) ----
-      float nl = 0.f, sc = 0.f;
+      float nl = 0.f;  // e^{-M} phi(q) z_t
       if (has_lin && ok) {
-        sc = ex2(-m_used);  // exp(-M), <= 1
+        const float sc = ex2(-m_used);  // exp(-M), <= 1
         const float* zp = p.z + bh * p.z_bh + t * p.z_t;
         const uint8_t* qrow = smem + C::OFF_Q + X * C::TILE_BYTES + r * 128;
 #pragma unroll
@@ -281,10 +286,13 @@ __global__ void __launch_bounds__(320, 1) hybrid_chunk_attn_kernel(const __grid_
               const float s0 = psi1(bf16lo(w[h]));
               const float s1 = psi1(bf16hi(w[h]));
               const int dim = 64 * b + 8 * cc + 2 * h;
-              nl += s0 * zp[dim] + (s0 * s0) * zp[D + dim] + s1 * zp[dim + 1] +
-                    (s1 * s1) * zp[D + dim + 1];
-              pa[cc * 4 + h] = pack_bf16(s0 * sc, s1 * sc);
-              pb[cc * 4 + h] = pack_bf16((s0 * s0) * sc, (s1 * s1) * sc);
+              const uint32_t ua = pack_bf16(s0 * sc, s1 * sc);
+              const uint32_t ub = pack_bf16((s0 * s0) * sc, (s1 * s1) * sc);
+              // n^L e^{-M} from the same bf16 features the phi~ S MMA uses
+              nl += bf16lo(ua) * zp[dim] + bf16hi(ua) * zp[dim + 1] + bf16lo(ub) * zp[D + dim] +
+                    bf16hi(ub) * zp[D + dim + 1];
+              pa[cc * 4 + h] = ua;
+              pb[cc * 4 + h] = ub;
             }
           }
           // features psi (0..D-1) then psi^2 (D..2D-1), two per column
@@ -300,7 +308,7 @@ __global__ void __launch_bounds__(320, 1) hybrid_chunk_attn_kernel(const __grid_
 
       if (ok) {
         if (!PARTS) {
-          const float inv = 1.f / (l + (has_lin ? nl * sc : 0.f));
+          const float inv = 1.f / (l + nl);
 #pragma unroll
           for (int a = 0; a < D / 32; ++a) {
             uint32_t ov[32];
@@ -340,7 +348,7 @@ __global__ void __launch_bounds__(320, 1) hybrid_chunk_attn_kernel(const __grid_
                                      __uint_as_float(ov[4 * c + 2]), __uint_as_float(ov[4 * c + 3]));
             }
           }
-          if (vrow) p.nL[grow] = has_lin ? nl * sc : 0.f;
+          if (vrow) p.nL[grow] = nl;
         }
       }
     }
@@ -597,12 +605,13 @@ __global__ void __launch_bounds__(192, 1) phi_state_kernel(const __grid_constant
 #pragma unroll
           for (int h = 0; h < 4; ++h) {
             const float s0 = psi1(bf16lo(w[h])), s1 = psi1(bf16hi(w[h]));
-            za[2 * h] += s0;
-            za[2 * h + 1] += s1;
-            zb[2 * h] += s0 * s0;
-            zb[2 * h + 1] += s1 * s1;
             va[h] = pack_bf16(s0, s1);
             vb[h] = pack_bf16(s0 * s0, s1 * s1);
+            // sum phi(K) over the same bf16 features the phi(K)^T V MMA uses
+            za[2 * h] += bf16lo(va[h]);
+            za[2 * h + 1] += bf16hi(va[h]);
+            zb[2 * h] += bf16lo(vb[h]);
+            zb[2 * h + 1] += bf16hi(vb[h]);
           }
           pa = make_uint4(va[0], va[1], va[2], va[3]);
           pb = make_uint4(vb[0], vb[1], vb[2], vb[3]);

@@ -35,8 +35,17 @@ def max_over_rms(y, ref):
     return float(np.abs(y - ref).max() / np.sqrt((ref ** 2).mean()))
 
 
-def assert_bf16_close(y, ref, what=""):
-    e2, em = rel_l2(y, ref), max_over_rms(y, ref)
+def assert_bf16_close(y, ref, what="", rowwise=False):
+    """rowwise: the max-abs bound is taken against each row's own RMS (for
+    inputs whose rows differ in magnitude by >10x, where rounding the exact
+    result to bf16 alone exceeds 3e-2 of the global RMS)."""
+    e2 = rel_l2(y, ref)
+    if rowwise:
+        y = np.asarray(y, dtype=np.float64)
+        ref = np.asarray(ref, dtype=np.float64)
+        em = float((np.abs(y - ref) / np.sqrt((ref ** 2).mean(axis=-1, keepdims=True))).max())
+    else:
+        em = max_over_rms(y, ref)
     assert e2 <= BF16_L2 and em <= BF16_MAX, f"{what}: rel L2 {e2:.3e}, max/RMS {em:.3e}"
     return e2, em
 
@@ -122,7 +131,13 @@ BF16_CASES = [
     (1, 1, 128, 1, 77, 3, 1, 36),     # one short frame (single 77-row tile)
     (1, 1, 128, 9, 40, 2, 1, 37),     # short frames, many chunks
     (1, 1, 64, 3, 300, 1, 1, 38),     # 300-row chunks (a lone 44-row tile B)
+    (1, 1, 128, 300, 1, 2, 1, 39),    # one-token frames: 2-row chunks, 3-key windows
+    (1, 1, 64, 50, 3, 1, 5, 42),      # overlap 5x the chunk, 3-token frames
 ]
+# With 1-3 tokens per frame the first chunk's rows are a softmax over a few
+# keys (|y| ~ |v|) while later rows average hundreds of keys (|y| ~ 0.05):
+# bf16 output rounding of the large rows alone is ~0.035 of the global RMS.
+ROWWISE = {39, 42}
 
 
 @pytest.mark.parametrize("B,H,d,F,S,Tc,To,seed", BF16_CASES)
@@ -130,18 +145,21 @@ def test_forward_bf16_matches_oracle(B, H, d, F, S, Tc, To, seed):
     q, k, v = inputs.make_qkv(B, H, F * S, d, seed, rms_qk=True)
     y = R.forward(q.cuda(), k.cuda(), v.cuda(), F, S, Tc, To)
     ref = orc.oracle_forward(q, k, v, F, S, Tc, To)
-    assert_bf16_close(np64(y), ref)
+    assert_bf16_close(np64(y), ref, rowwise=seed in ROWWISE)
 
 
 @pytest.mark.parametrize("post", [(8.0, 1.0, 1.0), (3.0, 1.0, 1.0), (0.25, 0.25, 1.0)])
 def test_forward_bf16_softmax_and_linear_balance(post):
     """Scaled queries move the balance between the branches: q x 8 makes the
     softmax window dominate every chunk, q x 3 mixes both, q,k x 0.25 makes
-    scores flat so the linear term dominates."""
+    scores flat so the linear term dominates.  In these skewed inputs row
+    magnitudes differ by ~20x (sharp softmax rows ~ single v rows, linear rows
+    ~ averages), so bf16 output rounding alone exceeds 3e-2 of the *global*
+    RMS; the max-abs bound is applied per row against that row's RMS."""
     B, H, d, F, S, Tc, To = 1, 2, 128, 5, 160, 2, 1
     q, k, v = inputs.make_qkv(B, H, F * S, d, 40, rms_qk=True, post=post)
-    y = R.forward(q.cuda(), k.cuda(), v.cuda(), F, S, Tc, To)
-    assert_bf16_close(np64(y), orc.oracle_forward(q, k, v, F, S, Tc, To), str(post))
+    y = np64(R.forward(q.cuda(), k.cuda(), v.cuda(), F, S, Tc, To))
+    assert_bf16_close(y, orc.oracle_forward(q, k, v, F, S, Tc, To), str(post), rowwise=True)
 
 
 def test_forward_parts_match_oracle_parts():
@@ -155,9 +173,10 @@ def test_forward_parts_match_oracle_parts():
     lin = onL > 0
     assert (nL[~lin] == 0).all() and (aL[~lin] == 0).all()
     rows = lin[0, 0]
-    assert_bf16_close((aL / nL[..., None])[:, :, rows], (oL / onL[..., None])[:, :, rows], "linear branch")
-    mix = (nS / nL)[lin]
-    omix = (onS / onL)[lin]
+    assert_bf16_close(aL[:, :, rows] / nL[:, :, rows, None], oL[:, :, rows] / onL[:, :, rows, None],
+                      "linear branch")
+    mix = nS[lin] / nL[lin]
+    omix = onS[lin] / onL[lin]
     assert np.abs(mix / omix - 1).max() < 2e-3
     y = (aS + aL) / (nS + nL)[..., None]
     assert_bf16_close(y, orc.oracle_forward(q, k, v, F, S, Tc, To), "recombined")
@@ -193,29 +212,35 @@ def test_forward_capi_and_stages_agree_bitwise():
     assert torch.equal(a, b) and torch.equal(a, c) and torch.equal(a, d2)
 
 
-def test_step_bf16_streamed_matches_forward_and_oracle():
-    B, H, d, F, S, Tc, To = 1, 2, 128, 8, 120, 3, 1
+def stream_steps(qd, kd, vd, F, S, Tc, To, Sst, zst, capi_every=2, workspace=None, outs=None):
+    """Feed a video through rehyat_step chunk by chunk; returns the outputs."""
+    res = []
+    t = 0
+    while t * min(Tc, F) < F:
+        f0, w, cf, qf, ef = R.step_frames(t, F, Tc, To)
+        o = None if outs is None else outs[t]
+        res.append(R.step(qd[:, :, f0 * S:(f0 + qf) * S].contiguous(), kd[:, :, w * S:(f0 + qf) * S].contiguous(),
+                          vd[:, :, w * S:(f0 + qf) * S].contiguous(), Sst, zst, S, qf, cf, ef, out=o,
+                          workspace=workspace, capi=(capi_every > 0 and t % capi_every == 1)))
+        t += 1
+    return res, t
+
+
+@pytest.mark.parametrize("F,S,Tc,To", [(8, 120, 3, 1), (7, 64, 2, 3), (6, 50, 1, 0)])
+def test_step_bf16_streamed_matches_forward_and_oracle(F, S, Tc, To):
+    B, H, d = 1, 2, 128
     q, k, v = inputs.make_qkv(B, H, F * S, d, 70, rms_qk=True)
     qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
     Sst = torch.zeros(B, H, 2 * d, d, device="cuda")
     zst = torch.zeros(B, H, 2 * d, device="cuda")
-    outs = []
-    t = 0
-    while t * Tc < F:
-        f0, w, cf, qf, ef = R.step_frames(t, F, Tc, To)
-        outs.append(R.step(qd[:, :, f0 * S:(f0 + qf) * S].contiguous(), kd[:, :, w * S:(f0 + qf) * S].contiguous(),
-                           vd[:, :, w * S:(f0 + qf) * S].contiguous(), Sst, zst, S, qf, cf, ef, capi=(t % 2 == 1)))
-        t += 1
+    outs, nsteps = stream_steps(qd, kd, vd, F, S, Tc, To, Sst, zst)
     y = np64(torch.cat(outs, dim=2))
     ref = orc.oracle_forward(q, k, v, F, S, Tc, To)
     assert_bf16_close(y, ref, "step vs oracle")
     yf = np64(R.forward(qd, kd, vd, F, S, Tc, To))
     assert rel_l2(y, yf) <= 5e-3
-    # the carried state equals the sum over every folded key
-    So, zo = orc.oracle_chunk_states(k, v, F, S, Tc, To)
-    # after the last step the state covers [0, w_last + evicted) = all keys before
-    # the end of the video minus nothing left in the last window's tail
-    f0, w, cf, qf, ef = R.step_frames(t - 1, F, Tc, To)
+    # the carried state is the sum over every folded key
+    f0, w, cf, qf, ef = R.step_frames(nsteps - 1, F, Tc, To)
     n_fold = (w + ef) * S
     PK = orc.phi(k[:, :, :n_fold].double().numpy())
     S_ref = np.einsum("bhje,bhjc->bhec", PK, v[:, :, :n_fold].double().numpy())
@@ -269,3 +294,76 @@ def test_wan13b_480p_sampled_rows():
     rows = sample_rows(F, S, Tc)
     ref = orc.oracle_forward(q, k, v, F, S, Tc, To, rows=rows)
     assert_bf16_close(np64(y[:, :, rows]), ref)
+
+
+def _head_rows_check(y, q, k, v, F, S, Tc, To, heads, rows):
+    """Oracle on the given (b, h) heads and query rows only."""
+    for b, h in heads:
+        ref = orc.oracle_forward(q[b:b + 1, h:h + 1], k[b:b + 1, h:h + 1], v[b:b + 1, h:h + 1], F, S, Tc, To,
+                                 rows=rows)
+        assert_bf16_close(np64(y[b:b + 1, h:h + 1, rows]), ref, f"head {(b, h)}")
+
+
+def few_rows(F, S, Tc, edge=32, n_rand=128, seed=7):
+    """Edges of the first, second, middle and last chunk plus random rows."""
+    N = F * S
+    Np = min(Tc, F) * S
+    nc = -(-F // min(Tc, F))
+    rows = set()
+    for t in sorted({0, min(1, nc - 1), nc // 2, nc - 1}):
+        q0, q1 = t * Np, min((t + 1) * Np, N)
+        rows.update(range(q0, min(q0 + edge, q1)))
+        rows.update(range(max(q1 - edge, q0), q1))
+    rows.update(np.random.default_rng(seed).integers(0, N, n_rand).tolist())
+    return np.array(sorted(rows))
+
+
+def test_wan14b_720p_sampled_rows():
+    """B=1, H=40, d=128, F=21 x 3600 tokens (75,600), T_c=3, T_o=1."""
+    B, H, d, F, S, Tc, To = 1, 40, 128, 21, 3600, 3, 1
+    q, k, v = inputs.make_qkv(B, H, F * S, d, 3, rms_qk=True)
+    y = R.forward(q.cuda(), k.cuda(), v.cuda(), F, S, Tc, To).cpu()
+    _head_rows_check(y, q, k, v, F, S, Tc, To, [(0, 0), (0, 17), (0, 39)], few_rows(F, S, Tc))
+
+
+def test_recurrent_81_frames_streamed_flat_memory():
+    """F=81 x 1560 tokens streamed through rehyat_step (27 chunks, T_c=3,
+    T_o=1): parity against the oracle on sampled rows, agreement with the
+    parallel form, and device memory flat across steps."""
+    B, H, d, F, S, Tc, To = 1, 12, 128, 81, 1560, 3, 1
+    q, k, v = inputs.make_qkv(B, H, F * S, d, 2, rms_qk=True)
+    qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+    Sst = torch.zeros(B, H, 2 * d, d, device="cuda")
+    zst = torch.zeros(B, H, 2 * d, device="cuda")
+    nc = -(-F // Tc)
+    outs = [torch.empty(B, H, R.step_frames(t, F, Tc, To)[3] * S, d, dtype=torch.bfloat16, device="cuda")
+            for t in range(nc)]
+    ws = R.alloc_workspace(R.step_workspace_bytes(B, H, S, d, Tc, To, Tc), qd.device)
+    chunks = []
+    for t in range(nc):
+        f0, w, cf, qf, ef = R.step_frames(t, F, Tc, To)
+        chunks.append((qd[:, :, f0 * S:(f0 + qf) * S].contiguous(), kd[:, :, w * S:(f0 + qf) * S].contiguous(),
+                       vd[:, :, w * S:(f0 + qf) * S].contiguous(), qf, cf, ef))
+    torch.cuda.synchronize()
+    torch.cuda.reset_peak_memory_stats()
+    base = torch.cuda.memory_allocated()
+    for (qc, kc, vc, qf, cf, ef), o in zip(chunks, outs):
+        R.step(qc, kc, vc, Sst, zst, S, qf, cf, ef, out=o, workspace=ws)
+    torch.cuda.synchronize()
+    assert torch.cuda.max_memory_allocated() == base, "step allocated device memory"
+    y = torch.cat(outs, dim=2).cpu()
+    rows = few_rows(F, S, Tc, edge=16, n_rand=64)
+    _head_rows_check(y, q, k, v, F, S, Tc, To, [(0, 0), (0, 11)], rows)
+    yf = R.forward(qd, kd, vd, F, S, Tc, To).cpu()
+    assert rel_l2(np64(y), np64(yf)) <= 5e-3
+
+
+@pytest.mark.parametrize("F", [21, 41, 81, 161])
+@pytest.mark.parametrize("Tc,To", [(2, 1), (3, 1), (5, 2)])
+def test_scaling_sweep_points_sampled(F, Tc, To):
+    """B=2, H=12, d=128, 1560 tokens/frame: every sweep point, two heads."""
+    B, H, d, S = 2, 12, 128, 1560
+    seed = 100 + [(2, 1), (3, 1), (5, 2)].index((Tc, To)) * 4 + [21, 41, 81, 161].index(F)
+    q, k, v = inputs.make_qkv(B, H, F * S, d, seed, rms_qk=True)
+    y = R.forward(q.cuda(), k.cuda(), v.cuda(), F, S, Tc, To).cpu()
+    _head_rows_check(y, q, k, v, F, S, Tc, To, [(0, 3), (1, 11)], few_rows(F, S, Tc, edge=16, n_rand=64))
