@@ -138,6 +138,32 @@ int rehyat_chunk_states(const void* k, const void* v,
                         int chunk_frames, int overlap_frames,
                         float* S, float* z, void* stream);
 
+/* rehyat_forward for callers that cannot allocate device memory during a
+ * call (no counterpart in the paper: it is a deployment variant).  Examples:
+ * a serving process that reserves all GPU memory at start-up and forbids
+ * later allocation, because cudaMalloc may synchronise the device and has
+ * unbounded latency; a plugin whose host framework owns the allocator and
+ * exposes no scratch hook.  The caller still passes q, k, v and out as for
+ * rehyat_forward; the scratch comes from a fixed array of
+ * REHYAT_NOALLOC_SCRATCH_BYTES inside the library, which every GPU that
+ * loads the library holds until the process exits.
+ *   - Allocates nothing: no cudaMalloc / cudaMallocAsync / cudaFree.
+ *   - When the default scratch layout does not fit, the key segments are
+ *     summed in fewer pieces (fewer CTAs, same result up to fp32 rounding
+ *     order); a problem that does not fit even then returns REHYAT_ENOMEM
+ *     before launching anything (1.3B-480p needs ~30 MB and fits).
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress, with that device current); make that first call
+ *     before any stream capture.
+ *   - All calls on a device share the one array: calls whose kernels overlap
+ *     on the GPU (different streams, no ordering) race and corrupt each
+ *     other; order them.  Each call writes every scratch byte it reads. */
+#define REHYAT_NOALLOC_SCRATCH_BYTES (32u << 20)
+int rehyat_forward_noalloc(const void* q, const void* k, const void* v,
+                           int B, int H, int F, int S_tok, int d,
+                           int chunk_frames, int overlap_frames,
+                           void* out, void* stream);
+
 /* ---------------------------------------------------------------------- *
  * Recurrent form (§3.3 chunk-wise RNN), one chunk per call.               *
  * ---------------------------------------------------------------------- */

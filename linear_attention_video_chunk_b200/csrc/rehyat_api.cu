@@ -534,3 +534,83 @@ REHYAT_API int rehyat_device_status(unsigned int* detail) {
   if (detail != nullptr) *detail = v;
   return v == 0 ? REHYAT_OK : REHYAT_ETIMEOUT;
 }
+
+// ===========================================================================
+// Forward without any allocation (scratch in a fixed device array)
+// ===========================================================================
+// Some callers cannot allocate device memory at call time: a serving process
+// that reserves all of the GPU's memory at start-up and forbids later
+// allocation (cudaMalloc can synchronise the device and its latency is
+// unbounded), or a plugin whose host framework owns the allocator and offers
+// no scratch hook.  rehyat_forward_noalloc serves them: its scratch lives in
+// the file-scope array below, which every GPU that loads this library holds
+// (REHYAT_NOALLOC_SCRATCH_BYTES each) until the process exits.
+//
+// In host code the name g_noalloc_scratch is only a host-side stand-in for
+// the device array, never a device address; the address is looked up with
+// cudaGetSymbolAddress once per device (on that device's first call, with the
+// device current) and only that address is handed to kernels and to TMA.
+namespace {
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[REHYAT_NOALLOC_SCRATCH_BYTES];
+
+constexpr int kMaxDevices = 128;
+std::mutex g_noalloc_mu;
+void* g_noalloc_addr[kMaxDevices] = {};
+
+// Device address of the scratch array on the current device.
+int noalloc_scratch(void** addr) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return REHYAT_ECUDA;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (g_noalloc_addr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) {
+      (void)cudaGetLastError();
+      return REHYAT_ECUDA;
+    }
+    g_noalloc_addr[dev] = p;
+  }
+  *addr = g_noalloc_addr[dev];
+  return REHYAT_OK;
+}
+
+// The forward's scratch layout with a given number of pieces per segment.
+size_t layout_with_nsplit(FwdPlan* P, int nsplit) {
+  P->nsplit = nsplit;
+  const size_t D2 = 2 * static_cast<size_t>(P->D);
+  const size_t segs = static_cast<size_t>(P->BH) * P->n_seg * nsplit;
+  const size_t chunks = static_cast<size_t>(P->BH) * P->nc;
+  size_t off = 0;
+  P->off_pS = off; off += align256(segs * D2 * P->D * 4);
+  P->off_pz = off; off += align256(segs * D2 * 4);
+  P->off_hi = off; off += align256(chunks * D2 * P->D * 2);
+  P->off_lo = off; off += align256(chunks * D2 * P->D * 2);
+  P->off_zt = off; off += align256(chunks * D2 * 4);
+  P->bytes = off > 0 ? off : 256;
+  return P->bytes;
+}
+
+}  // namespace
+
+REHYAT_API int rehyat_forward_noalloc(const void* q, const void* k, const void* v, int B, int H, int F, int S_tok,
+                                      int d, int chunk_frames, int overlap_frames, void* out, void* stream) {
+  FwdPlan P;
+  int st = plan_forward(B, H, F, S_tok, d, chunk_frames, overlap_frames, &P);
+  if (st != REHYAT_OK) return st;
+  if (check_qkvo(q, k, v, out)) return REHYAT_EINVAL;
+  // Fewer key pieces per segment shrink the partial sums until they fit.
+  int nsplit = P.nsplit;
+  while (layout_with_nsplit(&P, nsplit) > REHYAT_NOALLOC_SCRATCH_BYTES && nsplit > 1) --nsplit;
+  if (P.bytes > REHYAT_NOALLOC_SCRATCH_BYTES) return REHYAT_ENOMEM;  // problem too large for the array
+  void* ws = nullptr;
+  st = noalloc_scratch(&ws);
+  if (st != REHYAT_OK) return st;
+  // Every scratch byte this call reads is first written by this call, so
+  // nothing is cleared; calls that overlap on the GPU share the array and race.
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  st = run_states(k, v, P, w, nullptr, nullptr, s);
+  if (st != REHYAT_OK) return st;
+  return run_attention(q, k, v, P, w, out, nullptr, nullptr, nullptr, nullptr, nullptr, s);
+}

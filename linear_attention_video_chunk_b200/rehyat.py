@@ -35,6 +35,7 @@ _SIGS = {
     "rehyat_step_f32": [_vp, _vp, _vp, _vp, _vp, _vp, _I, _I, _I, _I, _I, _I, _I, _vp],
     "rehyat_phi": [_vp, _I, _vp, _I, ctypes.c_int64, _I, _vp],
     "rehyat_device_status": [ctypes.POINTER(ctypes.c_uint)],
+    "rehyat_forward_noalloc": [_vp, _vp, _vp, _I, _I, _I, _I, _I, _I, _I, _vp, _vp],
 }
 _RESTYPES = {"rehyat_status_string": ctypes.c_char_p}
 
@@ -138,6 +139,22 @@ def forward_capi(q, k, v, F, S_tok, chunk_frames, overlap_frames, out=None):
     out = torch.empty_like(q) if out is None else out
     _check(lib().rehyat_forward(_p(q), _p(k), _p(v), B, H, F, S_tok, d, chunk_frames, overlap_frames, _p(out),
                                 _stream()), "rehyat_forward")
+    return out
+
+
+NOALLOC_SCRATCH_BYTES = 32 << 20
+
+
+def forward_noalloc(q, k, v, F, S_tok, chunk_frames, overlap_frames, out):
+    """rehyat_forward_noalloc: the forward with no device allocation at all
+    (scratch in a fixed array inside the library; ``out`` must be given).
+    For callers that cannot allocate during a call; calls on one device must
+    not overlap on the GPU (they share the array)."""
+    for n, t in (("q", q), ("k", k), ("v", v), ("out", out)):
+        _need(t, torch.bfloat16, n)
+    B, H, N, d = _shape(q, F, S_tok)
+    _check(lib().rehyat_forward_noalloc(_p(q), _p(k), _p(v), B, H, F, S_tok, d, chunk_frames, overlap_frames,
+                                        _p(out), _stream()), "rehyat_forward_noalloc")
     return out
 
 
