@@ -215,6 +215,12 @@ int rehyat_step_f32(const float* q_c, const float* k_c, const float* v_c,
 int rehyat_phi(const void* x, int x_dtype, void* y, int y_dtype,
                int64_t rows, int d, void* stream);
 
+/* Diagnostic: y[i] = 2^x[i] by the FMA-pipe exponential the fused kernel uses
+ * for part of its softmax weights (round-to-nearest range reduction and a
+ * fitted cubic; max relative error 7.5e-5 for x in [-125, 8]; x < -125 is
+ * treated as -125).  x, y: n floats in device memory. */
+int rehyat_exp2_fma(const float* x, float* y, int64_t n, void* stream);
+
 /* Synchronises the current device and reports whether any kernel of this
  * library recorded a device-side error since the last call (REHYAT_ETIMEOUT
  * when a bounded wait ran out), then clears the record.  *detail (optional)

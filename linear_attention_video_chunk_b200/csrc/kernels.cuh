@@ -30,6 +30,7 @@ struct AttnParams {
   float* aL;
   float* nL;
   float* Mo;
+  unsigned long long* trace;  // clock64 stamps, only with -DREHYAT_TRACE (else unused)
 };
 
 // phi(K)^T V and sum phi(K) over key segments (tensor cores).  One CTA =
@@ -83,6 +84,9 @@ cudaError_t launch_state_accumulate(const float* part_S, const float* part_z, in
 // fp32 state -> bf16 hi/lo pair.
 cudaError_t launch_state_split(const float* S, long long n, __nv_bfloat16* hi, __nv_bfloat16* lo,
                                cudaStream_t s);
+
+// The FMA-pipe exp2 used for part of the softmax exponentials (diagnostic).
+cudaError_t launch_exp2_fma(const float* x, float* y, long long n, cudaStream_t s);
 
 cudaError_t launch_attention_f32(const AttnF32Params& p, int n_chunks, cudaStream_t s);
 cudaError_t launch_chunk_state_f32(const StateF32Params& p, cudaStream_t s);

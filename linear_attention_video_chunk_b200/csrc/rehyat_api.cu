@@ -19,7 +19,9 @@ cudaError_t read_and_clear_device_error(unsigned int* v);
 namespace {
 using namespace rehyat;
 
-constexpr int kSplitTarget = 296;  // CTAs aimed at for the state kernels (2 waves of 148 SMs)
+// CTAs aimed at for the state kernels: one wave of B200's 148 SMs (a
+// constant, so the fp32 summation order does not depend on the device).
+constexpr int kSplitTarget = 148;
 
 // ---------------------------------------------------------------------------
 // validation
@@ -67,8 +69,8 @@ int plan_forward(int B, int H, int F, int S_tok, int d, int Tc, int To, FwdPlan*
   p->n_seg = p->nc - 1;
   const int max_tiles = cdiv(p->chunk_tok, 64);
   p->nsplit = 1;
-  if (p->n_seg > 0) {
-    const long long want = (kSplitTarget + BH * p->n_seg - 1) / (BH * p->n_seg);
+  if (p->n_seg > 0) {  // pieces per segment: at most one wave of CTAs
+    const long long want = kSplitTarget / (BH * p->n_seg);
     p->nsplit = static_cast<int>(want < 1 ? 1 : (want > max_tiles ? max_tiles : want));
   }
   p->pairs = cdiv(cdiv(p->chunk_tok, 128), 2);
@@ -118,7 +120,7 @@ int plan_step(int B, int H, int S_tok, int d, int qf, int cf, int ef, StepPlan* 
   p->Nk = static_cast<int>(Nk);
   p->evict_tok = ef * S_tok;
   const int max_tiles = cdiv(p->evict_tok > 0 ? p->evict_tok : 1, 64);
-  const long long want = (kSplitTarget + BH - 1) / BH;
+  const long long want = kSplitTarget / BH;
   p->nsplit = static_cast<int>(want < 1 ? 1 : (want > max_tiles ? max_tiles : want));
   p->pairs = cdiv(cdiv(p->Nq, 128), 2);
   const long long units = BH * p->pairs;
@@ -176,6 +178,10 @@ bool make_map(CUtensorMap* m, const void* base, long long inner, long long rows,
 
 int cuda_status(cudaError_t e) { return e == cudaSuccess ? REHYAT_OK : REHYAT_ECUDA; }
 
+#ifdef REHYAT_TRACE
+unsigned long long* g_trace = nullptr;  // cycle-trace buffer of trace builds
+#endif
+
 // ---------------------------------------------------------------------------
 // stages
 // ---------------------------------------------------------------------------
@@ -223,6 +229,9 @@ int run_attention(const void* q, const void* k, const void* v, const FwdPlan& P,
   ap.z_t = 2LL * P.D;
   ap.out = static_cast<__nv_bfloat16*>(out);
   ap.aS = aS; ap.nS = nS; ap.aL = aL; ap.nL = nL; ap.Mo = Mo;
+#ifdef REHYAT_TRACE
+  ap.trace = g_trace;
+#endif
   return cuda_status(launch_attention(P.D, aS != nullptr, ap, P.n_units, s));
 }
 
@@ -527,6 +536,11 @@ REHYAT_API int rehyat_phi(const void* x, int x_dtype, void* y, int y_dtype, int6
                                 static_cast<cudaStream_t>(stream)));
 }
 
+REHYAT_API int rehyat_exp2_fma(const float* x, float* y, int64_t n, void* stream) {
+  if (x == nullptr || y == nullptr || n < 1) return REHYAT_EINVAL;
+  return cuda_status(launch_exp2_fma(x, y, n, static_cast<cudaStream_t>(stream)));
+}
+
 REHYAT_API int rehyat_device_status(unsigned int* detail) {
   unsigned int v = 0;
   if (cudaDeviceSynchronize() != cudaSuccess) return REHYAT_ECUDA;
@@ -614,3 +628,8 @@ REHYAT_API int rehyat_forward_noalloc(const void* q, const void* k, const void* 
   if (st != REHYAT_OK) return st;
   return run_attention(q, k, v, P, w, out, nullptr, nullptr, nullptr, nullptr, nullptr, s);
 }
+
+#ifdef REHYAT_TRACE
+// Trace builds only: where the fused kernel writes its cycle stamps.
+REHYAT_API void rehyat_trace_buffer(void* buf) { g_trace = static_cast<unsigned long long*>(buf); }
+#endif

@@ -40,6 +40,65 @@ __device__ __forceinline__ float psi1(float x) {  // 1 + elu(x)
   return x > 0.f ? x + 1.f : ex2(x * kLog2e);
 }
 
+// 2^x on the FMA/ALU pipes, for the share of softmax exponentials taken off
+// the SFU.  Range reduction: n = round(x) by adding 1.5 * 2^23 (the rounding
+// happens in the fp32 add), f = x - n in [-0.5, 0.5]; 2^f by a cubic whose
+// coefficients were fitted here to minimise relative error (Chebyshev-node
+// least squares with Lawson reweighting); n is then added to the result's
+// exponent field.  Max relative error in fp32 over [-125, 8]: 7.5e-5, far
+// below the 2^-9 of the bf16 P it feeds.  x < -125 is clamped (2^-125 stands
+// in for ~0); callers never pass -inf.
+__device__ __forceinline__ float exp2_fma(float x) {
+  x = fmaxf(x, -125.f);
+  const float t = x + 12582912.f;
+  const float f = x - (t - 12582912.f);
+  const float p = fmaf(fmaf(fmaf(0x1.c3f748p-5f, f, 0x1.f0de1ap-3f), f, 0x1.62f31ap-1f), f, 0x1.fff692p-1f);
+  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+}
+
+#ifndef REHYAT_EXP2_FMA_MASK
+// Columns c of each score tile with bit (c % 8) set take exp2_fma instead
+// of ex2 (0x11 = 2 of 8).  Measured on B200 at the Wan2.1-1.3B shape, any
+// share made the kernel slower (the softmax is latency-bound, not SFU-bound),
+// so the default is none.
+#define REHYAT_EXP2_FMA_MASK 0x00u
+#endif
+
+// P = 2^(s * scale - m) for one half (64 keys) of a 128-key row tile, packed
+// to bf16 pairs and stored into TMEM columns [32*HALF, 32*HALF + 32) of S;
+// returns the row sum of exactly the stored bf16 values.
+template <uint32_t FMA_MASK, int HALF>
+__device__ __forceinline__ float exp_pack_store(uint32_t (&s)[4][32], float scale, float neg_m, uint32_t tS) {
+  float rsum[4] = {0.f, 0.f, 0.f, 0.f};  // independent partial sums
+  uint32_t pk[32];
+#pragma unroll
+  for (int a = 2 * HALF; a < 2 * HALF + 2; ++a) {
+#pragma unroll
+    for (int c = 0; c < 16; ++c) {
+      const float x0 = fmaf(__uint_as_float(s[a][2 * c]), scale, neg_m);
+      const float x1 = fmaf(__uint_as_float(s[a][2 * c + 1]), scale, neg_m);
+      const float p0 = ((FMA_MASK >> ((2 * c) & 7)) & 1u) ? exp2_fma(x0) : ex2(x0);
+      const float p1 = ((FMA_MASK >> ((2 * c + 1) & 7)) & 1u) ? exp2_fma(x1) : ex2(x1);
+      const uint32_t u = pack_bf16(p0, p1);
+      // the denominator sums exactly the bf16 weights the P.V MMA uses
+      float& acc = rsum[c & 3];
+      acc = add_bf16_hi(u, add_bf16_lo(u, acc));
+      pk[(a & 1) * 16 + c] = u;
+    }
+  }
+  tmem_st32(tS + 32 * HALF, pk);
+  return (rsum[0] + rsum[1]) + (rsum[2] + rsum[3]);
+}
+
+// Make this warp's TMEM stores visible to the MMA issuer and arrive once on
+// `bar` for the whole warp.
+__device__ __forceinline__ void warp_release(uint32_t bar, int lane) {
+  tmem_st_wait();
+  tc_fence_before();
+  __syncwarp();
+  if (lane == 0) mbar_arrive(bar);
+}
+
 // ============================================================================
 // Fused chunk attention
 // ============================================================================
@@ -59,7 +118,7 @@ struct AttnCfg {
   static constexpr int B_FULL = 1;
   static constexpr int B_EMPTY = B_FULL + NSLOTS;
   static constexpr int B_S = B_EMPTY + NSLOTS;   // [2] scores ready in TMEM
-  static constexpr int B_P = B_S + 2;            // [2] probabilities written to TMEM
+  static constexpr int B_P = B_S + 2;            // [2] P written to TMEM
   static constexpr int B_O = B_P + 2;            // [2] last P.V done
   static constexpr int B_PHI = B_O + 2;          // [2] scaled phi(Q) written to TMEM
   static constexpr int B_LIN = B_PHI + 2;        // [2] linear MMA done
@@ -69,12 +128,42 @@ struct AttnCfg {
   static_assert(SMEM <= 232448, "shared memory");
   // TMEM columns: S/P of tile X at X*128, O of tile X at 256 + X*D.
   static constexpr uint32_t TMEM_COLS = 512;
+  // 12 warps: warpgroups 0 and 1 run the softmax of query tiles A and B,
+  // warpgroup 2 holds the TMA producer (warp 8) and the MMA issuer (warp 9).
+  // Launched at 168 registers a thread (65536 / 384, rounded down to 8);
+  // warpgroup 2 gives registers to the softmax warpgroups:
+  // 2 * 128 * REGS_SOFTMAX + 128 * REGS_ISSUE == 384 * REGS_LAUNCH.
+  static constexpr int THREADS = 384;
+  static constexpr uint32_t REGS_LAUNCH = 168;
+  static constexpr uint32_t REGS_SOFTMAX = 208;
+  static constexpr uint32_t REGS_ISSUE = 88;
+  static_assert(2 * 128 * REGS_SOFTMAX + 128 * REGS_ISSUE == THREADS * REGS_LAUNCH, "register split");
   static constexpr uint32_t IDESC_S = idesc_bf16_f32(128, 128, 0, 0);  // Q K^T: both K-major
   static constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, D, 0, 1);   // P V, phi~ S: B MN-major
 };
 
+// Optional cycle tracing (build with -DREHYAT_TRACE): CTAs 0..TRACE_CTAS-1
+// record clock64() at each stage of the first TRACE_TILES key tiles into
+// p.trace[cta][event][tile]; without the macro the hooks compile to nothing.
+#ifdef REHYAT_TRACE
+constexpr int TRACE_CTAS = 4, TRACE_EVENTS = 16, TRACE_TILES = 64;
+#define TRACE(ev, j)                                                                                  \
+  do {                                                                                               \
+    if (p.trace != nullptr && blockIdx.x < TRACE_CTAS && (j) < TRACE_TILES)                          \
+      p.trace[(blockIdx.x * TRACE_EVENTS + (ev)) * TRACE_TILES + (j)] = clock64();                   \
+  } while (0)
+#else
+#define TRACE(ev, j) \
+  do {               \
+  } while (0)
+#endif
+// events: softmax of tile X (lane 0 of warp 4X): 0+5X S ready seen, 1+5X S in
+// registers, 2+5X max done, 3+5X P stored, 4+5X P released; MMA issuer:
+// 10+X P_X seen, 12+X S_X(j+1) issued, 14 unit start (j = 0), Q and K_0 in
+// (j = 1), K_{j+1} in (j + 2), 15 P_A.V_j issued
+
 template <int D, bool PARTS>
-__global__ void __launch_bounds__(320, 1) hybrid_chunk_attn_kernel(const __grid_constant__ AttnParams p) {
+__global__ void __launch_bounds__(384, 1) hybrid_chunk_attn_kernel(const __grid_constant__ AttnParams p) {
   using C = AttnCfg<D>;
   constexpr int NS = C::NSLOTS;
   extern __shared__ uint8_t smem_raw[];
@@ -118,9 +207,9 @@ __global__ void __launch_bounds__(320, 1) hybrid_chunk_attn_kernel(const __grid_
     }
     for (int x = 0; x < 2; ++x) {
       mbar_init(BAR(C::B_S + x), 1);
-      mbar_init(BAR(C::B_P + x), 128);
+      mbar_init(BAR(C::B_P + x), 4);           // one arrive per softmax warp
       mbar_init(BAR(C::B_O + x), 1);
-      mbar_init(BAR(C::B_PHI + x), 128);
+      mbar_init(BAR(C::B_PHI + x), 4);
       mbar_init(BAR(C::B_LIN + x), 1);
     }
     mbar_init(BAR(C::B_FIN), 1);
@@ -151,6 +240,10 @@ __global__ void __launch_bounds__(320, 1) hybrid_chunk_attn_kernel(const __grid_
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const bool has_lin = (*lin_flag) != 0;
+  if (warp < 8)
+    regs_increase<C::REGS_SOFTMAX>();
+  else
+    regs_decrease<C::REGS_ISSUE>();
 
   if (warp < 8) {
     // ======================= softmax / epilogue warps =======================
@@ -171,6 +264,7 @@ __global__ void __launch_bounds__(320, 1) hybrid_chunk_attn_kernel(const __grid_
       for (int j = 0; j < ntiles; ++j) {
         ok = warp_wait(BAR(C::B_S + X), j & 1, abort);
         if (!ok) break;
+        if (wl == 0 && lane == 0) TRACE(0 + 5 * X, j);
         tc_fence_after();
         uint32_t s[4][32];
         tmem_ld32(tS + 0, s[0]);
@@ -182,6 +276,7 @@ __global__ void __launch_bounds__(320, 1) hybrid_chunk_attn_kernel(const __grid_
         reg_fence(s[1]);
         reg_fence(s[2]);
         reg_fence(s[3]);
+        if (wl == 0 && lane == 0) TRACE(1 + 5 * X, j);
         const int valid = win - j * 128;  // keys of this tile inside the window
         if (valid < 128) {                 // only the window's last tile is partial
 #pragma unroll
@@ -190,12 +285,21 @@ __global__ void __launch_bounds__(320, 1) hybrid_chunk_attn_kernel(const __grid_
             for (int c = 0; c < 32; ++c)
               if (a * 32 + c >= valid) s[a][c] = __float_as_uint(-INFINITY);
         }
-        float mraw = -INFINITY;  // scale > 0, so the max is taken on raw scores
+        // Row max on raw scores (scale > 0): eight independent chains of
+        // three-input max, then a short tree.
+        float mr[8];
 #pragma unroll
-        for (int a = 0; a < 4; ++a)
+        for (int i = 0; i < 8; ++i) {
+          const int a = i >> 1, c0 = (i & 1) * 16;
+          float m = fmax3(__uint_as_float(s[a][c0]), __uint_as_float(s[a][c0 + 1]), __uint_as_float(s[a][c0 + 2]));
 #pragma unroll
-          for (int c = 0; c < 32; ++c) mraw = fmaxf(mraw, __uint_as_float(s[a][c]));
+          for (int c = 3; c < 15; c += 2)
+            m = fmax3(m, __uint_as_float(s[a][c0 + c]), __uint_as_float(s[a][c0 + c + 1]));
+          mr[i] = fmaxf(m, __uint_as_float(s[a][c0 + 15]));
+        }
+        const float mraw = fmaxf(fmax3(fmax3(mr[0], mr[1], mr[2]), fmax3(mr[3], mr[4], mr[5]), mr[6]), mr[7]);
         const float mx = mraw * p.scale_log2;
+        if (wl == 0 && lane == 0) TRACE(2 + 5 * X, j);
         // Lazy rescaling: move the shift only when the row maximum exceeds
         // it by more than 2^8, so P <= 256 and fp32 sums stay exact enough.
         const bool need = mx > m_used + 8.f;
@@ -204,24 +308,12 @@ __global__ void __launch_bounds__(320, 1) hybrid_chunk_attn_kernel(const __grid_
         const float alpha = need ? ex2(m_used - mnew) : 1.f;
         m_used = mnew;
         const float neg_m = -m_used;
-        float rs = 0.f;
-        uint32_t pk[2][32];
-#pragma unroll
-        for (int a = 0; a < 4; ++a) {
-#pragma unroll
-          for (int c = 0; c < 16; ++c) {
-            const float p0 = ex2(fmaf(__uint_as_float(s[a][2 * c]), p.scale_log2, neg_m));
-            const float p1 = ex2(fmaf(__uint_as_float(s[a][2 * c + 1]), p.scale_log2, neg_m));
-            const uint32_t u = pack_bf16(p0, p1);
-            // the denominator sums exactly the bf16 weights the P.V MMA uses
-            rs += bf16lo(u) + bf16hi(u);
-            pk[a >> 1][(a & 1) * 16 + c] = u;
-          }
-        }
-        l = l * alpha + rs;
-        // P (bf16, two per column) overwrites the first 64 columns of S.
-        tmem_st32(tS + 0, pk[0]);
-        tmem_st32(tS + 32, pk[1]);
+        // Full tiles may send a share of the exponentials to the FMA pipe;
+        // the window's partial last tile stays on ex2 (masked keys give 0).
+        float rs = (valid >= 128) ? exp_pack_store<REHYAT_EXP2_FMA_MASK, 0>(s, p.scale_log2, neg_m, tS)
+                                  : exp_pack_store<0u, 0>(s, p.scale_log2, neg_m, tS);
+        rs += (valid >= 128) ? exp_pack_store<REHYAT_EXP2_FMA_MASK, 1>(s, p.scale_log2, neg_m, tS)
+                             : exp_pack_store<0u, 1>(s, p.scale_log2, neg_m, tS);
         if (warp_need && j > 0) {
           // O holds tiles 0..j-1 (their P.V completed before S_j was
           // signalled) and must move to the new shift before P_j.V_j.
@@ -235,10 +327,12 @@ __global__ void __launch_bounds__(320, 1) hybrid_chunk_attn_kernel(const __grid_
             for (int c = 0; c < 32; ++c) ov[c] = __float_as_uint(__uint_as_float(ov[c]) * alpha);
             tmem_st32(tO + 32 * a, ov);
           }
+          tmem_st_wait();
         }
-        tmem_st_wait();
-        tc_fence_before();
-        mbar_arrive(BAR(C::B_P + X));
+        if (wl == 0 && lane == 0) TRACE(3 + 5 * X, j);
+        warp_release(BAR(C::B_P + X), lane);
+        if (wl == 0 && lane == 0) TRACE(4 + 5 * X, j);
+        l = l * alpha + rs;
       }
 
       if (ok) ok = warp_wait(BAR(C::B_O + X), 0, abort);
@@ -299,9 +393,7 @@ __global__ void __launch_bounds__(320, 1) hybrid_chunk_attn_kernel(const __grid_
           tmem_st32(tS + 32 * b, pa);
           tmem_st32(tS + D / 2 + 32 * b, pb);
         }
-        tmem_st_wait();
-        tc_fence_before();
-        mbar_arrive(BAR(C::B_PHI + X));
+        warp_release(BAR(C::B_PHI + X), lane);
         ok = warp_wait(BAR(C::B_LIN + X), 0, abort);
         tc_fence_after();
       }
@@ -386,7 +478,7 @@ __global__ void __launch_bounds__(320, 1) hybrid_chunk_attn_kernel(const __grid_
       drain_wait(BAR(C::B_Q), 0);
       for (uint32_t s2 = (seq > NS ? seq - NS : 0); s2 < seq; ++s2) drain_wait(BAR(C::B_FULL + s2 % NS), (s2 / NS) & 1);
     }
-  } else {
+  } else if (warp == 9) {
     // =============================== MMA issuer ==============================
     if (lane == 0) {
       const uint32_t qA = smem_u32(smem + C::OFF_Q);
@@ -394,31 +486,49 @@ __global__ void __launch_bounds__(320, 1) hybrid_chunk_attn_kernel(const __grid_
       const uint32_t ring = smem_u32(smem + C::OFF_RING);
       auto slot_addr = [&](uint32_t sq) { return ring + (sq % NS) * C::TILE_BYTES; };
       // Q K^T: A = Q tile, B = K tile, both K-major; K-step kk moves 32 B
-      // inside a 128-B swizzle row (box kk/4).
-      auto issue_S = [&](uint32_t d_tmem, uint32_t qa, uint32_t kb) {
+      // inside a 128-B swizzle row (box kk/4).  Descriptors: constant high
+      // word, low word = base + compile-time step (see desc_hi_sw128).
+      constexpr uint32_t HI_K = desc_hi_sw128(1024);    // K-major: SBO = 8 rows
+      constexpr uint32_t HI_MN = desc_hi_sw128(1024);   // MN-major: SBO = 8 K-rows
+      const uint32_t lo_qA = desc_lo(qA, 16), lo_qB = desc_lo(qB, 16);
+      auto issue_S = [&](uint32_t d_tmem, uint32_t lo_q, uint32_t kb) {
+        const uint32_t lo_k = desc_lo(kb, 16);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * C::BOX_BYTES + (kk & 3) * 32;
-          mma_ss(d_tmem, smem_desc_sw128(qa + off, 16, 1024), smem_desc_sw128(kb + off, 16, 1024),
-                 C::IDESC_S, kk > 0 ? 1u : 0u);
+          const uint32_t step = ((kk >> 2) * C::BOX_BYTES + (kk & 3) * 32) >> 4;
+          mma_ss(d_tmem, desc_join(lo_q + step, HI_K), desc_join(lo_k + step, HI_K), C::IDESC_S, kk > 0 ? 1u : 0u);
         }
       };
       // P V: A = P in TMEM (8 columns per 16 keys), B = V tile MN-major:
-      // 16 keys = 2048 B; the two 64-column boxes are BOX_BYTES apart.
-      auto issue_PV = [&](uint32_t d_tmem, uint32_t a_tmem, uint32_t vb, bool first) {
+      // 16 keys = 2048 B; the two 64-column boxes are BOX_BYTES apart (LBO).
+      auto issue_PV_half = [&](uint32_t d_tmem, uint32_t a_tmem, uint32_t vb, bool first, int half) {
+        const uint32_t lo_v = desc_lo(vb, C::BOX_BYTES);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_ts(d_tmem, a_tmem + kk * 8, smem_desc_sw128(vb + kk * 2048, C::BOX_BYTES, 1024), C::IDESC_PV,
+        for (int k4 = 0; k4 < 4; ++k4) {
+          const int kk = 4 * half + k4;
+          mma_ts(d_tmem, a_tmem + kk * 8, desc_join(lo_v + ((kk * 2048) >> 4), HI_MN), C::IDESC_PV,
                  (first && kk == 0) ? 0u : 1u);
+        }
       };
+      // O_X += P_X V_j once the softmax warps have released P_X
+      auto issue_PV = [&](int X, uint32_t vb, int j) -> bool {
+        if (!mbar_wait(BAR(C::B_P + X), j & 1, abort)) return false;
+        TRACE(10 + X, j);
+        tc_fence_after();
+        issue_PV_half(tmem + 256 + X * D, tmem + X * 128, vb, j == 0, 0);
+        issue_PV_half(tmem + 256 + X * D, tmem + X * 128, vb, j == 0, 1);
+        return true;
+      };
+      TRACE(14, 0);
       bool ok = mbar_wait(BAR(C::B_Q), 0, abort);
       ok = ok && mbar_wait(BAR(C::B_FULL + 0), 0, abort);  // K_0 is sequence 0
+      TRACE(14, 1);
       tc_fence_after();
       if (ok) {
-        issue_S(tmem + 0, qA, slot_addr(0));
+        issue_S(tmem + 0, lo_qA, slot_addr(0));
         mma_commit(BAR(C::B_S + 0));
         if (hasB) {
-          issue_S(tmem + 128, qB, slot_addr(0));
+          issue_S(tmem + 128, lo_qB, slot_addr(0));
           mma_commit(BAR(C::B_S + 1));
         }
         mma_commit(BAR(C::B_EMPTY + 0));
@@ -426,29 +536,28 @@ __global__ void __launch_bounds__(320, 1) hybrid_chunk_attn_kernel(const __grid_
       for (int j = 0; ok && j < ntiles; ++j) {
         const uint32_t vq = 2 * j + 1, kn = 2 * j + 2;
         const bool more = j + 1 < ntiles;
-        ok = mbar_wait(BAR(C::B_FULL + vq % NS), (vq / NS) & 1, abort) &&
-             mbar_wait(BAR(C::B_P + 0), j & 1, abort);
+        ok = mbar_wait(BAR(C::B_FULL + vq % NS), (vq / NS) & 1, abort) && issue_PV(0, slot_addr(vq), j);
         if (!ok) break;
-        tc_fence_after();
-        issue_PV(tmem + 256, tmem + 0, slot_addr(vq), j == 0);
+        TRACE(15, j);
         if (more) {
           ok = mbar_wait(BAR(C::B_FULL + kn % NS), (kn / NS) & 1, abort);
           if (!ok) break;
+          TRACE(14, j + 2);
           tc_fence_after();
-          issue_S(tmem + 0, qA, slot_addr(kn));
+          issue_S(tmem + 0, lo_qA, slot_addr(kn));
           mma_commit(BAR(C::B_S + 0));
+          TRACE(12, j);
         } else {
           mma_commit(BAR(C::B_O + 0));
         }
         if (hasB) {
-          ok = mbar_wait(BAR(C::B_P + 1), j & 1, abort);
+          ok = issue_PV(1, slot_addr(vq), j);
           if (!ok) break;
-          tc_fence_after();
-          issue_PV(tmem + 256 + D, tmem + 128, slot_addr(vq), j == 0);
           mma_commit(BAR(C::B_EMPTY + vq % NS));
           if (more) {
-            issue_S(tmem + 128, qB, slot_addr(kn));
+            issue_S(tmem + 128, lo_qB, slot_addr(kn));
             mma_commit(BAR(C::B_S + 1));
+            TRACE(13, j);
             mma_commit(BAR(C::B_EMPTY + kn % NS));
           } else {
             mma_commit(BAR(C::B_O + 1));
@@ -474,7 +583,7 @@ __global__ void __launch_bounds__(320, 1) hybrid_chunk_attn_kernel(const __grid_
               const uint32_t sa = slot_addr(s0 + part * C::SPP + kk / 8);
               const uint32_t acc = PARTS ? ((part | kk) != 0 ? 1u : 0u) : 1u;
               mma_ts(tmem + 256 + X * D, tmem + X * 128 + kk * 8,
-                     smem_desc_sw128(sa + (kk & 7) * 2048, C::BOX_BYTES, 1024), C::IDESC_PV, acc);
+                     desc_join(desc_lo(sa + (kk & 7) * 2048, C::BOX_BYTES), HI_MN), C::IDESC_PV, acc);
             }
           }
           mma_commit(BAR(C::B_LIN + X));
@@ -511,19 +620,23 @@ struct StCfg {
   static constexpr uint32_t TMEM_COLS = (HALVES * D <= 64) ? 64 : ((HALVES * D <= 128) ? 128 : 256);
   static constexpr int OFF_BAR = NST * STAGE;
   static constexpr int SMEM = OFF_BAR + 256 + 1024;
+  static constexpr int PHI_WARPS = 8;                 // warps 0-7: phi(K), sum phi(K), epilogue
+  static constexpr int PHI_THREADS = 32 * PHI_WARPS;
+  static constexpr int THREADS = PHI_THREADS + 64;    // + TMA producer (warp 8) + MMA issuer (warp 9)
   static constexpr int CH = D / 8;                    // 16-byte chunks per row
-  static constexpr int G = 128 / CH;                  // token groups over 128 threads
+  static constexpr int G = PHI_THREADS / CH;          // token groups
   static constexpr int TPG = 64 / G;                  // tokens per thread per tile
   static constexpr int B_KV = 0, B_PHI = NST, B_EMPTY = 2 * NST, B_ACC = 3 * NST, B_FIN = 3 * NST + 1;
   // A = phi(K)^T (features x tokens, features contiguous: MN-major),
   // B = V (tokens x D, D contiguous: MN-major).
   static constexpr uint32_t IDESC = idesc_bf16_f32(128, D, 1, 1);
   static_assert(SMEM <= 232448, "shared memory");
-  static_assert(G * CH == 128 && TPG * G == 64, "thread mapping");
+  static_assert(G * CH == PHI_THREADS && TPG * G == 64, "thread mapping");
+  static_assert(G * 2 * D * 4 <= STAGE, "z reduction scratch");
 };
 
 template <int D>
-__global__ void __launch_bounds__(192, 1) phi_state_kernel(const __grid_constant__ StateParams p) {
+__global__ void __launch_bounds__(StCfg<D>::THREADS, 1) phi_state_kernel(const __grid_constant__ StateParams p) {
   using C = StCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -553,7 +666,7 @@ __global__ void __launch_bounds__(192, 1) phi_state_kernel(const __grid_constant
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::NST; ++i) {
       mbar_init(BAR(C::B_KV + i), 1);
-      mbar_init(BAR(C::B_PHI + i), 128);
+      mbar_init(BAR(C::B_PHI + i), C::PHI_WARPS);
       mbar_init(BAR(C::B_EMPTY + i), 1);
     }
     mbar_init(BAR(C::B_ACC), 1);
@@ -561,11 +674,11 @@ __global__ void __launch_bounds__(192, 1) phi_state_kernel(const __grid_constant
     *abort = 0;
     fence_mbar_init();
   }
-  if (warp == 4 && lane == 0) {
+  if (warp == C::PHI_WARPS && lane == 0) {
     prefetch_tmap(&p.tm_k);
     prefetch_tmap(&p.tm_v);
   }
-  if (warp == 5) {
+  if (warp == C::PHI_WARPS + 1) {
     tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
     tmem_relinquish();
   }
@@ -574,7 +687,7 @@ __global__ void __launch_bounds__(192, 1) phi_state_kernel(const __grid_constant
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp < 4) {
+  if (warp < C::PHI_WARPS) {
     // ============ phi(K) into the MN-major A operand, sum phi(K) ============
     // phi atom bx (< NBOX) = psi of dims 64bx..64bx+63, atom NBOX+bx = psi^2:
     // byte-for-byte the same positions as the K box bx, so no re-layout.
@@ -608,10 +721,10 @@ __global__ void __launch_bounds__(192, 1) phi_state_kernel(const __grid_constant
             va[h] = pack_bf16(s0, s1);
             vb[h] = pack_bf16(s0 * s0, s1 * s1);
             // sum phi(K) over the same bf16 features the phi(K)^T V MMA uses
-            za[2 * h] += bf16lo(va[h]);
-            za[2 * h + 1] += bf16hi(va[h]);
-            zb[2 * h] += bf16lo(vb[h]);
-            zb[2 * h + 1] += bf16hi(vb[h]);
+            za[2 * h] = add_bf16_lo(va[h], za[2 * h]);
+            za[2 * h + 1] = add_bf16_hi(va[h], za[2 * h + 1]);
+            zb[2 * h] = add_bf16_lo(vb[h], zb[2 * h]);
+            zb[2 * h + 1] = add_bf16_hi(vb[h], zb[2 * h + 1]);
           }
           pa = make_uint4(va[0], va[1], va[2], va[3]);
           pb = make_uint4(vb[0], vb[1], vb[2], vb[3]);
@@ -620,44 +733,53 @@ __global__ void __launch_bounds__(192, 1) phi_state_kernel(const __grid_constant
         *reinterpret_cast<uint4*>(ph + (C::NBOX + bx) * C::BOX + off) = pb;
       }
       fence_proxy_async_smem();
-      mbar_arrive(BAR(C::B_PHI + st));
+      __syncwarp();
+      if (lane == 0) mbar_arrive(BAR(C::B_PHI + st));
     }
     // ---- epilogue: TMEM accumulators -> partial state rows ----
     if (ok) ok = mbar_wait(BAR(C::B_ACC), 0, abort);
     ok = __all_sync(kFull, ok);
     tc_fence_after();
+    // warps 0-3 and 4-7 cover the same TMEM lanes; split the work between
+    // them by feature half (two halves) or by column half (one half)
+    const int quarter = warp & 3, grp = warp >> 2;
+    const int h = (C::HALVES == 2) ? grp : 0;
+    constexpr int NCOL = (C::HALVES == 2) ? D : D / 2;
+    const int col0 = (C::HALVES == 2) ? 0 : grp * (D / 2);
     if (ok) {
+      const int e = 128 * h + 32 * quarter + lane;
 #pragma unroll
-      for (int h = 0; h < C::HALVES; ++h) {
-        const int e = 128 * h + 32 * warp + lane;
+      for (int q = 0; q < NCOL / 32; ++q) {
+        uint32_t v[32];
+        tmem_ld32(tmem + (static_cast<uint32_t>(32 * quarter) << 16) + h * D + col0 + 32 * q, v);
+        tmem_ld_wait();
+        reg_fence(v);
+        float4* dst = reinterpret_cast<float4*>(outS + static_cast<size_t>(e) * D + col0 + 32 * q);
 #pragma unroll
-        for (int q = 0; q < D / 32; ++q) {
-          uint32_t v[32];
-          tmem_ld32(tmem + (static_cast<uint32_t>(32 * warp) << 16) + h * D + 32 * q, v);
-          tmem_ld_wait();
-          reg_fence(v);
-          float4* dst = reinterpret_cast<float4*>(outS + static_cast<size_t>(e) * D + 32 * q);
-#pragma unroll
-          for (int k4 = 0; k4 < 8; ++k4)
-            dst[k4] = make_float4(__uint_as_float(v[4 * k4]), __uint_as_float(v[4 * k4 + 1]),
-                                  __uint_as_float(v[4 * k4 + 2]), __uint_as_float(v[4 * k4 + 3]));
-        }
+        for (int k4 = 0; k4 < 8; ++k4)
+          dst[k4] = make_float4(__uint_as_float(v[4 * k4]), __uint_as_float(v[4 * k4 + 1]),
+                                __uint_as_float(v[4 * k4 + 2]), __uint_as_float(v[4 * k4 + 3]));
       }
-      // sum phi(K) across the token groups (stage 0 is free: every MMA is done)
-      float* zred = reinterpret_cast<float*>(smem);
+    }
+    // sum phi(K) across the token groups (stage 0 is free once every MMA is
+    // done; the barrier is reached by all 256 threads whatever `ok` is)
+    float* zred = reinterpret_cast<float*>(smem);
+    if (ok) {
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
         zred[g * 2 * D + 8 * c + e] = za[e];
         zred[g * 2 * D + D + 8 * c + e] = zb[e];
       }
-      asm volatile("bar.sync 1, 128;" ::: "memory");
-      for (int f = tid; f < 2 * D; f += 128) {
+    }
+    asm volatile("bar.sync 1, %0;" ::"n"(C::PHI_THREADS) : "memory");
+    if (ok) {
+      for (int f = tid; f < 2 * D; f += C::PHI_THREADS) {
         float acc = 0.f;
         for (int gg = 0; gg < C::G; ++gg) acc += zred[gg * 2 * D + f];
         outz[f] = acc;
       }
     }
-  } else if (warp == 4) {
+  } else if (warp == C::PHI_WARPS) {
     // =============================== TMA producer ============================
     if (lane == 0) {
       bool ok = true;
@@ -705,7 +827,7 @@ __global__ void __launch_bounds__(192, 1) phi_state_kernel(const __grid_constant
 #undef BAR
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == C::PHI_WARPS + 1) {
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
   }
@@ -780,6 +902,12 @@ __global__ void state_split_kernel(const float* __restrict__ S, long long n, __n
   }
 }
 
+__global__ void exp2_fma_kernel(const float* __restrict__ x, float* __restrict__ y, long long n) {
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<long long>(gridDim.x) * blockDim.x)
+    y[i] = exp2_fma(x[i]);
+}
+
 int grid_for(long long n, int threads) {
   long long g = (n + threads - 1) / threads;
   if (g > 148LL * 16) g = 148LL * 16;
@@ -794,9 +922,15 @@ int state_smem_bytes(int D) { return D == 128 ? StCfg<128>::SMEM : StCfg<64>::SM
 template <int D, bool PARTS>
 static cudaError_t launch_attn_t(const AttnParams& p, int n_units, cudaStream_t s) {
   auto* k = hybrid_chunk_attn_kernel<D, PARTS>;
-  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, AttnCfg<D>::SMEM);
+  // The in-kernel register split assumes exactly REGS_LAUNCH registers per
+  // thread at launch; with fewer, a warpgroup's increase could never be met.
+  cudaFuncAttributes fa;
+  cudaError_t e = cudaFuncGetAttributes(&fa, k);
   if (e != cudaSuccess) return e;
-  k<<<n_units, 320, AttnCfg<D>::SMEM, s>>>(p);
+  if (static_cast<uint32_t>(fa.numRegs) != AttnCfg<D>::REGS_LAUNCH) return cudaErrorInvalidConfiguration;
+  e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, AttnCfg<D>::SMEM);
+  if (e != cudaSuccess) return e;
+  k<<<n_units, AttnCfg<D>::THREADS, AttnCfg<D>::SMEM, s>>>(p);
   return cudaGetLastError();
 }
 
@@ -811,7 +945,7 @@ static cudaError_t launch_state_t(const StateParams& p, int n_ctas, cudaStream_t
   auto* k = phi_state_kernel<D>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, StCfg<D>::SMEM);
   if (e != cudaSuccess) return e;
-  k<<<n_ctas, 192, StCfg<D>::SMEM, s>>>(p);
+  k<<<n_ctas, StCfg<D>::THREADS, StCfg<D>::SMEM, s>>>(p);
   return cudaGetLastError();
 }
 
@@ -833,6 +967,11 @@ cudaError_t launch_state_accumulate(const float* part_S, const float* part_z, in
                                     float* state_S, float* state_z, cudaStream_t s) {
   const long long n = static_cast<long long>(BH) * 2 * D * (D + 1);
   state_accumulate_kernel<<<grid_for(n, 256), 256, 0, s>>>(part_S, part_z, BH, nsplit, D, state_S, state_z);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_exp2_fma(const float* x, float* y, long long n, cudaStream_t s) {
+  exp2_fma_kernel<<<grid_for(n, 256), 256, 0, s>>>(x, y, n);
   return cudaGetLastError();
 }
 

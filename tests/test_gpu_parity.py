@@ -367,3 +367,15 @@ def test_scaling_sweep_points_sampled(F, Tc, To):
     q, k, v = inputs.make_qkv(B, H, F * S, d, seed, rms_qk=True)
     y = R.forward(q.cuda(), k.cuda(), v.cuda(), F, S, Tc, To).cpu()
     _head_rows_check(y, q, k, v, F, S, Tc, To, [(0, 3), (1, 11)], few_rows(F, S, Tc, edge=16, n_rand=64))
+
+
+def test_exp2_fma_error_bound():
+    """The FMA-pipe 2^x used for part of the softmax weights stays within its
+    stated relative error (7.5e-5) of the exact power over [-125, 8]."""
+    x = torch.cat([torch.linspace(-125.0, 8.0, 1_000_001),
+                   torch.rand(100_000, generator=torch.Generator().manual_seed(3)) * 133.0 - 125.0])
+    y = R.exp2_fma(x.cuda()).cpu().double().numpy()
+    ref = np.exp2(x.double().numpy())
+    assert np.abs(y / ref - 1).max() < 8e-5
+    lo = R.exp2_fma(torch.tensor([-200.0, -125.0], device="cuda")).cpu().double().numpy()
+    np.testing.assert_allclose(lo, [2.0 ** -125] * 2, rtol=1e-4)

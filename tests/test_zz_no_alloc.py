@@ -24,10 +24,15 @@ BF16_L2, BF16_MAX = 1e-2, 3e-2   # the bf16 tolerance of the other parity tests
 
 
 def _close(y, ref):
+    """(rel L2, max-abs / RMS) of y against ref.  Both are bf16 outputs of
+    the same computation whose fp32 sums ran in a different order (the array
+    version merges key pieces), so an element may round to the neighbouring
+    bf16 value: one bf16 ulp of |ref| is allowed before the max-abs term."""
     y = y.double().cpu().numpy()
     ref = ref.double().cpu().numpy()
     e2 = (np.sqrt(((y - ref) ** 2).sum((-2, -1))) / np.sqrt((ref ** 2).sum((-2, -1)))).max()
-    em = np.abs(y - ref).max() / np.sqrt((ref ** 2).mean())
+    ulp = np.exp2(np.floor(np.log2(np.maximum(np.abs(ref), 1e-30))) - 7)
+    em = np.maximum(np.abs(y - ref) - ulp, 0).max() / np.sqrt((ref ** 2).mean())
     return e2, em
 
 
@@ -49,6 +54,9 @@ def test_noalloc_matches_forward_on_two_calls_in_a_row():
         assert torch.isfinite(out.float()).all()
         e2, em = _close(out, ref)
         assert e2 <= BF16_L2 and em <= BF16_MAX, (seed, e2, em)
+        if R.workspace_bytes(B, H, F, S, d, Tc, To) <= R.NOALLOC_SCRATCH_BYTES:
+            # same scratch layout as rehyat_forward: same kernels, same order
+            assert torch.equal(out, ref)
     assert R.device_status() == R.OK
 
 
