@@ -53,13 +53,17 @@ def chunks(F, S, Tc, To):
         yield q0, q1, max(q0 - to * S, 0), q1
 
 
-def work(c):
+def work(c, sets="causal"):
     B, H, d, F, S, Tc, To = (c[k] for k in ("B", "H", "d", "F", "S_tok", "T_c", "T_o"))
     BH, N, D2 = B * H, F * S, 2 * d
     ch = list(chunks(F, S, Tc, To))
     pairs = sum((q1 - q0) * (hi - lo) for q0, q1, lo, hi in ch)
-    n_lin = sum(q1 - q0 for q0, q1, lo, hi in ch if lo > 0)       # queries with a linear term
-    folded = max(lo for _, _, lo, _ in ch)                        # keys folded into states
+    if sets == "causal":
+        n_lin = sum(q1 - q0 for q0, q1, lo, hi in ch if lo > 0)   # queries with a linear term
+        folded = max(lo for _, _, lo, _ in ch)                    # keys folded into states
+    else:
+        n_lin = sum(q1 - q0 for q0, q1, lo, hi in ch if lo > 0 or hi < N)
+        folded = N if len(ch) > 1 else 0
     attn_flops = BH * (4 * d * pairs + 2 * D2 * (d + 1) * n_lin)
     state_flops = BH * 2 * D2 * (d + 1) * folded
     attn_bytes = BH * N * d * 2 * 4 + BH * len(ch) * D2 * (d * 4 + 4)     # q,k,v,out + states (hi,lo,z)
@@ -212,13 +216,23 @@ def run_forward_bench(args, c, rank, world, dev):
     ws = R.alloc_workspace(R.workspace_bytes(B, H, F, S, d, Tc, To), dev)
     torch.cuda.synchronize()
 
+    if args.sets != "causal":  # one call (states + attention) per step
+        n = R.ctypes.c_size_t(0)
+        R.lib().rehyat_forward_ex_workspace_bytes(B, H, F, S, d, Tc, To, R.SETS[args.sets], R.ctypes.byref(n))
+        ws = R.alloc_workspace(n.value, dev)
+
     def step(e0=None, e1=None, e2=None):
         if e0 is not None:
             e0.record()
-        R.forward_states(kd, vd, F, S, Tc, To, ws)
-        if e1 is not None:
-            e1.record()
-        R.forward_attention(qd, kd, vd, F, S, Tc, To, out, ws)
+        if args.sets != "causal":
+            if e1 is not None:
+                e1.record()
+            R.forward_sets(qd, kd, vd, F, S, Tc, To, sets=args.sets, out=out, workspace=ws)
+        else:
+            R.forward_states(kd, vd, F, S, Tc, To, ws)
+            if e1 is not None:
+                e1.record()
+            R.forward_attention(qd, kd, vd, F, S, Tc, To, out, ws)
         if e2 is not None:
             e2.record()
 
@@ -249,10 +263,17 @@ def run_forward_bench(args, c, rank, world, dev):
                     h2d=0, d2h=0, q=q, k=k, v=v, launches=3 * K)
     out_h = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
     Ke = max(3, min(K, 20))
+
+    def fwd(o):  # the public API call a user makes
+        if args.sets == "causal":
+            R.forward(qd, kd, vd, F, S, Tc, To, out=o, workspace=ws)
+        else:
+            R.forward_sets(qd, kd, vd, F, S, Tc, To, sets=args.sets, out=o, workspace=ws)
+
     for _ in range(2):
         for src, dst in ((q, qd), (k, kd), (v, vd)):
             dst.copy_(src, non_blocking=True)
-        R.forward(qd, kd, vd, F, S, Tc, To, out=out, workspace=ws)
+        fwd(out)
         out_h.copy_(out, non_blocking=True)
     torch.cuda.synchronize()
     if world > 1:
@@ -262,7 +283,7 @@ def run_forward_bench(args, c, rank, world, dev):
     for _ in range(Ke):
         for src, dst in ((q, qd), (k, kd), (v, vd)):
             dst.copy_(src, non_blocking=True)
-        R.forward(qd, kd, vd, F, S, Tc, To, out=out, workspace=ws)
+        fwd(out)
         out_h.copy_(out, non_blocking=True)
     e2.record()
     torch.cuda.synchronize()
@@ -294,9 +315,11 @@ def run_ours(args):
         res = run_recurrent_bench(args, c, rank, world, dev)
     else:
         res = run_forward_bench(args, c, rank, world, dev)
-    w = work(c)
+    w = work(c, args.sets)
     bf16_peak, bf16_sus, hbm, src = peaks()
     tokens = w["tokens"] * world
+    if args.sets != "causal":
+        c["workload"] += f" ({args.sets} sets)"
     line = {
         "metric": METRIC, "value": tokens / (res["ms_step"] / 1e3), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": res["ms_step"], "higher_is_better": True,
@@ -307,7 +330,7 @@ def run_ours(args):
                    "tokens_per_step_per_gpu": w["tokens"], "parallelism": f"replicas x{world} (no collective)",
                    "l2": "inputs larger than L2: q+k+v = %.0f MB per GPU" % (3 * w["tokens"] * c["H"] * c["d"] * 2 / 1e6)},
     }
-    if args.config != "recurrent":
+    if args.config != "recurrent" and args.sets == "causal":
         achieved = w["attn_flops"] / (res["attn_ms"] / 1e3) / 1e12
         line["roofline"] = {
             "kernel": "hybrid_chunk_attn_kernel", "bound": "tensor", "achieved": achieved, "peak": bf16_peak,
@@ -322,7 +345,14 @@ def run_ours(args):
                    "d2h_bytes_per_step": res["d2h"], "ms_per_step": res["e2e_ms"]}
     line["clocks"] = res["clocks"]
     line["gpu_launches"] = res["launches"]
-    if rank == 0 and world == 1 and not args.no_cpu_baseline and args.config == "wan13b" and not args.heads:
+    if args.sets != "causal":  # one call per step: the path's fraction is the figure
+        line["roofline"] = {"kernel": "whole path (states + fused attention)", "bound": "tensor",
+                            "achieved": (w["attn_flops"] + w["state_flops"]) / (res["ms_step"] / 1e3) / 1e12,
+                            "peak": bf16_peak, "unit": "TFLOP/s", "traffic": None,
+                            "peak_source": f"{src} bf16 dense (burst)"}
+        line["roofline"]["frac"] = line["roofline"]["achieved"] / bf16_peak
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and args.config == "wan13b" and not args.heads \
+            and args.sets == "causal":
         rate, n, dt = oracle_sample_rate(c, res["q"], res["k"], res["v"], args.cpu_budget)
         line["cpu_baseline"] = {"value": rate, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
                                 "sample": f"fp64 explicit-mask oracle on {n} random query rows x all {c['H']} "
@@ -374,6 +404,53 @@ def run_recurrent_bench(args, c, rank, world, dev):
         torch.cuda.synchronize()
     ms = max_over_ranks(s0.elapsed_time(s1) / K, world, dev)
     return dict(ms_step=ms, e2e_ms=ms, clocks=clk.summary(), h2d=0, d2h=0, launches=K * nc * 4, q=q, k=k, v=v)
+
+
+def run_compare_full(args):
+    """The hybrid against full bidirectional softmax over the same tokens:
+    our fused kernel with one chunk covering every frame (pure softmax), and
+    torch's scaled_dot_product_attention as a library reference; FLOPs are
+    the algorithmic counts of each computation."""
+    import torch
+    from linear_attention_video_chunk_b200 import inputs
+    from linear_attention_video_chunk_b200 import rehyat as R
+    dev = torch.device("cuda", 0)
+    bf16_peak, _, _, src = peaks()
+    B, H, d, F, S = 1, 12, 128, 21, 1560
+    q, k, v = (x.to(dev) for x in inputs.make_qkv(B, H, F * S, d, 1, rms_qk=True))
+    out = torch.empty_like(q)
+
+    def timed(fn, K=10):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(K):
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / K
+
+    rows = []
+    for Tc, To in ((F, 0), (1, 0), (1, 1), (2, 1), (3, 0), (3, 1), (3, 2), (5, 2), (7, 1)):
+        ws = R.alloc_workspace(R.workspace_bytes(B, H, F, S, d, Tc, To), dev)
+        ms = timed(lambda: R.forward(q, k, v, F, S, Tc, To, out=out, workspace=ws))
+        w = work(dict(B=B, H=H, d=d, F=F, S_tok=S, T_c=Tc, T_o=To))
+        fl = w["attn_flops"] + w["state_flops"]
+        rows.append({"T_c": Tc, "T_o": To, "kind": "full softmax (one chunk)" if Tc >= F else "hybrid",
+                     "ms": ms, "tflop": fl / 1e12, "tflops_per_s": fl / (ms / 1e3) / 1e12,
+                     "frac_of_peak": fl / (ms / 1e3) / 1e12 / bf16_peak})
+    sdpa = torch.nn.functional.scaled_dot_product_attention
+    ms = timed(lambda: sdpa(q, k, v))
+    fl = B * H * 4 * d * (F * S) ** 2
+    rows.append({"kind": "torch scaled_dot_product_attention (library, full softmax)", "ms": ms,
+                 "tflop": fl / 1e12, "tflops_per_s": fl / (ms / 1e3) / 1e12})
+    full = rows[0]["ms"]
+    for r in rows:
+        r["speedup_vs_full"] = full / r["ms"]
+        print(json.dumps({"compare_full": r, "workload": "Wan2.1-1.3B 480p shape",
+                          "peak": f"{bf16_peak} TFLOP/s {src}"}), flush=True)
 
 
 def run_sweep(args):
@@ -469,6 +546,8 @@ def main():
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--config", choices=tuple(CONFIGS), default="wan13b")
     ap.add_argument("--sweep", action="store_true")
+    ap.add_argument("--compare-full", action="store_true", help="hybrid vs full softmax over (T_c, T_o)")
+    ap.add_argument("--sets", choices=("causal", "bidirectional"), default="causal")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end leg (profiling runs)")
     ap.add_argument("--heads", type=int, default=0, help="override H (smaller profiling cases)")
@@ -480,6 +559,8 @@ def main():
         run_reference(args)
     elif args.sweep:
         run_sweep(args)
+    elif args.compare_full:
+        run_compare_full(args)
     else:
         run_ours(args)
 

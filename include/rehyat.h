@@ -21,7 +21,8 @@
  *     D' = 2d): the only concrete psi the paper gives.
  *   - softmax weight exp(q.k / sqrt(d)).
  *   - every call computes the §3.3 (causal / recurrent) sets, so the parallel
- *     form and the step form compute the same function.
+ *     form and the step form compute the same function; rehyat_forward_ex
+ *     also offers the §3.2 bidirectional sets.
  *
  * Conventions for every entry point:
  *   - Tensors are dense, row-major, in DEVICE memory owned by the caller:
@@ -108,6 +109,25 @@ int rehyat_forward_attention(const void* q, const void* k, const void* v,
                              int chunk_frames, int overlap_frames,
                              void* out, void* workspace, size_t workspace_bytes,
                              void* stream);
+
+/* Set modes of rehyat_forward_ex. */
+#define REHYAT_SETS_CAUSAL 0        /* §3.3 recurrent sets: T^L_t = { j < lo_t } (rehyat_forward) */
+#define REHYAT_SETS_BIDIRECTIONAL 1 /* §3.2 sets with overlap: T^L_t = T - T^S_t (earlier and later keys) */
+
+/* rehyat_forward with a choice of sets.  REHYAT_SETS_BIDIRECTIONAL is the
+ * non-causal variant (§3.2 sets with overlap; the causal vs non-causal
+ * comparison of §5.3): chunk t's linear term covers every key outside its
+ * softmax window [lo_t, min((t+1)N', N)), later keys included, so it has no
+ * recurrent form.  workspace may be NULL (then stream-ordered scratch is
+ * allocated and freed on `stream`), else it must hold
+ * rehyat_forward_ex_workspace_bytes(..., sets) bytes, 256-byte aligned. */
+int rehyat_forward_ex_workspace_bytes(int B, int H, int F, int S_tok, int d,
+                                      int chunk_frames, int overlap_frames, int sets,
+                                      size_t* bytes);
+int rehyat_forward_ex(const void* q, const void* k, const void* v,
+                      int B, int H, int F, int S_tok, int d,
+                      int chunk_frames, int overlap_frames, int sets,
+                      void* out, void* workspace, size_t workspace_bytes, void* stream);
 
 /* fp32 forward (SIMT fp32 throughout, accurate exp); same sets and layout.
  * Meant for small problems and tight-tolerance checks; any size is legal. */

@@ -11,6 +11,10 @@
 // The linear state entering chunk t is the sum over [0, lo_t).  It is built
 // from "segments": segment s covers keys [lo_s, lo_{s+1}), so the state of
 // chunk t is the exclusive prefix over segments 0 .. t-1.
+//
+// With the §3.2 bidirectional sets (T^L_t = T - T^S_t) the state of chunk t
+// is the sum over every key outside [lo_t, hi_t); segments are then single
+// frames and the state is prefix(lo_t) + suffix(hi_t).
 #pragma once
 
 #include <cstdint>
@@ -60,10 +64,16 @@ struct SegGeom {
   int nsplit;     // CTAs per segment (token ranges split evenly)
   int step;       // 1: a single segment [0, step_tok)
   int step_tok;
+  int seg_tok;    // > 0: fixed segments [s * seg_tok, (s + 1) * seg_tok) (one frame each)
 
   RH_HD void seg(int s, int& a, int& b) const {
     if (step) {
       a = 0; b = step_tok;
+      return;
+    }
+    if (seg_tok > 0) {
+      a = imin(s * seg_tok, N_k);
+      b = imin(a + seg_tok, N_k);
       return;
     }
     a = imin(imax(s * chunk_tok - ovl_tok, 0), N_k);

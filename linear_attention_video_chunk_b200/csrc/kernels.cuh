@@ -78,6 +78,10 @@ cudaError_t launch_chunk_state(int D, const StateParams& p, int n_ctas, cudaStre
 cudaError_t launch_state_scan(const float* part_S, const float* part_z, int BH, int n_seg,
                               int nsplit, int n_chunks, int D, __nv_bfloat16* hi,
                               __nv_bfloat16* lo, float* Sf, float* zt, cudaStream_t s);
+// Bidirectional sets: per-frame partials -> prefix(lo_t) + suffix(hi_t).
+cudaError_t launch_state_scan_bidir(const float* part_S, const float* part_z, int BH, int F, int nsplit,
+                                    int n_chunks, int D, int Tc, int To, __nv_bfloat16* hi, __nv_bfloat16* lo,
+                                    float* Sf, float* zt, cudaStream_t s);
 // state_S/z += sum over pieces of one segment's partials.
 cudaError_t launch_state_accumulate(const float* part_S, const float* part_z, int BH, int nsplit,
                                     int D, float* state_S, float* state_z, cudaStream_t s);

@@ -45,6 +45,7 @@ size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
 struct FwdPlan {
   int BH, N, D, nc, n_seg, nsplit, chunk_tok, ovl_tok, pairs, n_units;
+  int F, S_tok, tc, to, bidir;  // bidir: §3.2 sets (frame segments, prefix + suffix states)
   size_t off_pS, off_pz, off_hi, off_lo, off_zt, bytes;       // bf16 path
   size_t f32_off_pS, f32_off_pz, f32_off_S, f32_off_zt, f32_bytes;  // fp32 path
 };
@@ -63,6 +64,11 @@ int plan_forward(int B, int H, int F, int S_tok, int d, int Tc, int To, FwdPlan*
   p->BH = static_cast<int>(BH);
   p->N = static_cast<int>(N);
   p->D = d;
+  p->F = F;
+  p->S_tok = S_tok;
+  p->tc = tc;
+  p->to = to;
+  p->bidir = 0;
   p->chunk_tok = tc * S_tok;
   p->ovl_tok = to * S_tok;
   p->nc = cdiv(F, tc);
@@ -95,6 +101,34 @@ int plan_forward(int B, int H, int F, int S_tok, int d, int Tc, int To, FwdPlan*
   p->f32_off_zt = off; off += align256(chunks * D2 * 4);
   p->f32_bytes = off;
   if (p->nc > 65535 || p->BH > 65535) p->f32_bytes = 0;  // fp32 grids use y/z dims
+  return REHYAT_OK;
+}
+
+// Plan for the chosen sets.  The bidirectional sets sum keys per frame (so
+// that both window edges are segment edges); the attention is unchanged.
+int plan_forward_sets(int B, int H, int F, int S_tok, int d, int Tc, int To, int sets, FwdPlan* p) {
+  if (sets != REHYAT_SETS_CAUSAL && sets != REHYAT_SETS_BIDIRECTIONAL) return REHYAT_EINVAL;
+  int st = plan_forward(B, H, F, S_tok, d, Tc, To, p);
+  if (st != REHYAT_OK || sets == REHYAT_SETS_CAUSAL) return st;
+  p->bidir = 1;
+  p->n_seg = (p->nc > 1) ? F : 0;  // one chunk: the complement of its window is empty
+  p->nsplit = 1;
+  if (p->n_seg > 0) {
+    const long long want = kSplitTarget / (static_cast<long long>(p->BH) * p->n_seg);
+    const int max_tiles = cdiv(S_tok, 64);
+    p->nsplit = static_cast<int>(want < 1 ? 1 : (want > max_tiles ? max_tiles : want));
+  }
+  if (static_cast<long long>(p->BH) * p->n_seg * p->nsplit > INT_MAX) return REHYAT_EINVAL;
+  const size_t D2 = 2 * static_cast<size_t>(d);
+  const size_t segs = static_cast<size_t>(p->BH) * p->n_seg * p->nsplit;
+  const size_t chunks = static_cast<size_t>(p->BH) * p->nc;
+  size_t off = 0;
+  p->off_pS = off; off += align256(segs * D2 * d * 4);
+  p->off_pz = off; off += align256(segs * D2 * 4);
+  p->off_hi = off; off += align256(chunks * D2 * d * 2);
+  p->off_lo = off; off += align256(chunks * D2 * d * 2);
+  p->off_zt = off; off += align256(chunks * D2 * 4);
+  p->bytes = off > 0 ? off : 256;
   return REHYAT_OK;
 }
 
@@ -194,12 +228,23 @@ int run_states(const void* k, const void* v, const FwdPlan& P, uint8_t* ws, floa
     std::memset(&sp, 0, sizeof(sp));
     if (!make_map(&sp.tm_k, k, P.D, P.N, P.BH, 64) || !make_map(&sp.tm_v, v, P.D, P.N, P.BH, 64))
       return REHYAT_ECUDA;
-    sp.sg = SegGeom{P.N, P.chunk_tok, P.ovl_tok, P.n_seg, P.nsplit, 0, 0};
+    sp.sg = SegGeom{P.N, P.chunk_tok, P.ovl_tok, P.n_seg, P.nsplit, 0, 0, P.bidir ? P.S_tok : 0};
     sp.BH = P.BH;
     sp.part_S = pS;
     sp.part_z = pz;
     int st = cuda_status(launch_chunk_state(P.D, sp, P.BH * P.n_seg * P.nsplit, s));
     if (st != REHYAT_OK) return st;
+  }
+  if (P.bidir) {
+    if (P.n_seg == 0)  // one chunk: no linear set; the causal scan writes zero states
+      return cuda_status(launch_state_scan(pS, pz, P.BH, 0, 1, P.nc, P.D,
+                                           Sf_out ? nullptr : reinterpret_cast<__nv_bfloat16*>(ws + P.off_hi),
+                                           Sf_out ? nullptr : reinterpret_cast<__nv_bfloat16*>(ws + P.off_lo), Sf_out,
+                                           Sf_out ? z_out : reinterpret_cast<float*>(ws + P.off_zt), s));
+    return cuda_status(launch_state_scan_bidir(pS, pz, P.BH, P.F, P.nsplit, P.nc, P.D, P.tc, P.to,
+                                               Sf_out ? nullptr : reinterpret_cast<__nv_bfloat16*>(ws + P.off_hi),
+                                               Sf_out ? nullptr : reinterpret_cast<__nv_bfloat16*>(ws + P.off_lo),
+                                               Sf_out, Sf_out ? z_out : reinterpret_cast<float*>(ws + P.off_zt), s));
   }
   if (Sf_out != nullptr)
     return cuda_status(launch_state_scan(pS, pz, P.BH, P.n_seg, P.nsplit, P.nc, P.D, nullptr, nullptr, Sf_out,
@@ -333,6 +378,39 @@ REHYAT_API int rehyat_forward(const void* q, const void* k, const void* v, int B
   st = ws.alloc(P.bytes);
   if (st != REHYAT_OK) return st;
   return rehyat_forward_ws(q, k, v, B, H, F, S_tok, d, chunk_frames, overlap_frames, out, ws.p, P.bytes, stream);
+}
+
+REHYAT_API int rehyat_forward_ex_workspace_bytes(int B, int H, int F, int S_tok, int d, int chunk_frames,
+                                                 int overlap_frames, int sets, size_t* bytes) {
+  if (bytes == nullptr) return REHYAT_EINVAL;
+  FwdPlan P;
+  int st = plan_forward_sets(B, H, F, S_tok, d, chunk_frames, overlap_frames, sets, &P);
+  if (st != REHYAT_OK) return st;
+  *bytes = P.bytes;
+  return REHYAT_OK;
+}
+
+REHYAT_API int rehyat_forward_ex(const void* q, const void* k, const void* v, int B, int H, int F, int S_tok, int d,
+                                 int chunk_frames, int overlap_frames, int sets, void* out, void* workspace,
+                                 size_t workspace_bytes, void* stream) {
+  FwdPlan P;
+  int st = plan_forward_sets(B, H, F, S_tok, d, chunk_frames, overlap_frames, sets, &P);
+  if (st != REHYAT_OK) return st;
+  if (check_qkvo(q, k, v, out)) return REHYAT_EINVAL;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  WsGuard own(s);
+  if (workspace == nullptr) {
+    st = own.alloc(P.bytes);
+    if (st != REHYAT_OK) return st;
+    workspace = own.p;
+  } else {
+    if (reinterpret_cast<uintptr_t>(workspace) % 256 != 0) return REHYAT_EINVAL;
+    if (workspace_bytes < P.bytes) return REHYAT_ENOMEM;
+  }
+  uint8_t* w = static_cast<uint8_t*>(workspace);
+  st = run_states(k, v, P, w, nullptr, nullptr, s);
+  if (st != REHYAT_OK) return st;
+  return run_attention(q, k, v, P, w, out, nullptr, nullptr, nullptr, nullptr, nullptr, s);
 }
 
 REHYAT_API int rehyat_forward_parts(const void* q, const void* k, const void* v, int B, int H, int F, int S_tok,

@@ -103,6 +103,18 @@ def test_ws_variants_check_workspace(lib):
     assert lib.rehyat_forward_ws(16, 16, 16, 1, 1, 4, 8, 64, 2, 1, 16, 272, 1 << 30, None) == R.EINVAL
 
 
+def test_forward_ex_validation(lib):
+    f = lambda sets, ws=0, nb=0: lib.rehyat_forward_ex(16, 16, 16, 1, 1, 4, 8, 64, 2, 1, sets, 16, ws, nb, None)
+    assert f(2) == R.EINVAL              # unknown set mode
+    assert f(-1) == R.EINVAL
+    assert f(1, ws=256, nb=1) == R.ENOMEM  # workspace too small (checked before launching)
+    assert f(1, ws=272, nb=1 << 30) == R.EINVAL  # misaligned workspace
+    n0, n1 = ctypes.c_size_t(0), ctypes.c_size_t(0)
+    assert lib.rehyat_forward_ex_workspace_bytes(1, 12, 21, 1560, 128, 3, 1, 0, ctypes.byref(n0)) == R.OK
+    assert lib.rehyat_forward_ex_workspace_bytes(1, 12, 21, 1560, 128, 3, 1, 1, ctypes.byref(n1)) == R.OK
+    assert n0.value == R.workspace_bytes(1, 12, 21, 1560, 128, 3, 1) and n1.value > 0
+
+
 def test_phi_validation(lib):
     assert lib.rehyat_phi(0, 0, 16, 0, 4, 64, None) == R.EINVAL
     assert lib.rehyat_phi(16, 3, 16, 0, 4, 64, None) == R.EINVAL

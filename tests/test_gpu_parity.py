@@ -379,3 +379,40 @@ def test_exp2_fma_error_bound():
     assert np.abs(y / ref - 1).max() < 8e-5
     lo = R.exp2_fma(torch.tensor([-200.0, -125.0], device="cuda")).cpu().double().numpy()
     np.testing.assert_allclose(lo, [2.0 ** -125] * 2, rtol=1e-4)
+
+
+# --------------------------------------------------------------------------- #
+# bidirectional (§3.2) sets                                                    #
+# --------------------------------------------------------------------------- #
+BIDIR_CASES = [
+    # B, H, d, F, S_tok, Tc, To, seed
+    (1, 2, 128, 5, 200, 2, 1, 130),   # ragged: chunks with earlier and later linear keys
+    (1, 2, 64, 7, 90, 2, 3, 131),     # overlap longer than a chunk
+    (2, 1, 128, 6, 100, 3, 0, 132),   # no overlap: the §3.2 sets without overlap
+    (1, 1, 128, 3, 150, 4, 1, 133),   # one chunk: no linear set at all (full softmax)
+    (1, 1, 128, 9, 40, 1, 1, 134),    # one-frame chunks
+]
+
+
+@pytest.mark.parametrize("B,H,d,F,S,Tc,To,seed", BIDIR_CASES)
+def test_forward_bidirectional_matches_oracle(B, H, d, F, S, Tc, To, seed):
+    q, k, v = inputs.make_qkv(B, H, F * S, d, seed, rms_qk=True)
+    y = R.forward_sets(q.cuda(), k.cuda(), v.cuda(), F, S, Tc, To, sets="bidirectional")
+    ref = orc.oracle_forward(q, k, v, F, S, Tc, To, mode="bidirectional")
+    assert_bf16_close(np64(y), ref, "bidirectional")
+
+
+def test_forward_ex_causal_is_rehyat_forward():
+    B, H, d, F, S, Tc, To = 1, 2, 128, 6, 130, 3, 1
+    q, k, v = (x.cuda() for x in inputs.make_qkv(B, H, F * S, d, 135, rms_qk=True))
+    assert torch.equal(R.forward_sets(q, k, v, F, S, Tc, To, sets="causal"), R.forward(q, k, v, F, S, Tc, To))
+
+
+def test_wan13b_480p_bidirectional_sampled_rows():
+    """The non-causal variant at the Wan2.1-1.3B 480p shape (every head)."""
+    B, H, d, F, S, Tc, To = 1, 12, 128, 21, 1560, 3, 1
+    q, k, v = inputs.make_qkv(B, H, F * S, d, 1, rms_qk=True)
+    y = R.forward_sets(q.cuda(), k.cuda(), v.cuda(), F, S, Tc, To, sets="bidirectional").cpu()
+    rows = few_rows(F, S, Tc)
+    ref = orc.oracle_forward(q, k, v, F, S, Tc, To, mode="bidirectional", rows=rows)
+    assert_bf16_close(np64(y[:, :, rows]), ref, "bidirectional 1.3B")
