@@ -211,12 +211,14 @@ def run_forward_bench(args, c, rank, world, dev):
     B, H, d, F, S, Tc, To = (c[k] for k in ("B", "H", "d", "F", "S_tok", "T_c", "T_o"))
     N = F * S
     q, k, v = inputs.make_qkv(B, H, N, d, c["seed"] + 1000 * rank, rms_qk=True, pin=True)
+    if args.layout == "bnhd":  # heads interleaved per token: [B, N, H, d]
+        q, k, v = (x.transpose(1, 2).contiguous().pin_memory() for x in (q, k, v))
     qd, kd, vd = (x.to(dev, non_blocking=True) for x in (q, k, v))
     out = torch.empty_like(qd)
     ws = R.alloc_workspace(R.workspace_bytes(B, H, F, S, d, Tc, To), dev)
     torch.cuda.synchronize()
 
-    if args.sets != "causal":  # one call (states + attention) per step
+    if args.sets != "causal" or args.layout != "bhnd":  # one call (states + attention) per step
         n = R.ctypes.c_size_t(0)
         R.lib().rehyat_forward_ex_workspace_bytes(B, H, F, S, d, Tc, To, R.SETS[args.sets], R.ctypes.byref(n))
         ws = R.alloc_workspace(n.value, dev)
@@ -224,10 +226,10 @@ def run_forward_bench(args, c, rank, world, dev):
     def step(e0=None, e1=None, e2=None):
         if e0 is not None:
             e0.record()
-        if args.sets != "causal":
+        if args.sets != "causal" or args.layout != "bhnd":
             if e1 is not None:
                 e1.record()
-            R.forward_sets(qd, kd, vd, F, S, Tc, To, sets=args.sets, out=out, workspace=ws)
+            R.forward_sets(qd, kd, vd, F, S, Tc, To, sets=args.sets, layout=args.layout, out=out, workspace=ws)
         else:
             R.forward_states(kd, vd, F, S, Tc, To, ws)
             if e1 is not None:
@@ -265,10 +267,10 @@ def run_forward_bench(args, c, rank, world, dev):
     Ke = max(3, min(K, 20))
 
     def fwd(o):  # the public API call a user makes
-        if args.sets == "causal":
+        if args.sets == "causal" and args.layout == "bhnd":
             R.forward(qd, kd, vd, F, S, Tc, To, out=o, workspace=ws)
         else:
-            R.forward_sets(qd, kd, vd, F, S, Tc, To, sets=args.sets, out=o, workspace=ws)
+            R.forward_sets(qd, kd, vd, F, S, Tc, To, sets=args.sets, layout=args.layout, out=o, workspace=ws)
 
     for _ in range(2):
         for src, dst in ((q, qd), (k, kd), (v, vd)):
@@ -320,6 +322,8 @@ def run_ours(args):
     tokens = w["tokens"] * world
     if args.sets != "causal":
         c["workload"] += f" ({args.sets} sets)"
+    if args.layout != "bhnd":
+        c["workload"] += " ([B, N, H, d] layout)"
     line = {
         "metric": METRIC, "value": tokens / (res["ms_step"] / 1e3), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": res["ms_step"], "higher_is_better": True,
@@ -330,7 +334,7 @@ def run_ours(args):
                    "tokens_per_step_per_gpu": w["tokens"], "parallelism": f"replicas x{world} (no collective)",
                    "l2": "inputs larger than L2: q+k+v = %.0f MB per GPU" % (3 * w["tokens"] * c["H"] * c["d"] * 2 / 1e6)},
     }
-    if args.config != "recurrent" and args.sets == "causal":
+    if args.config != "recurrent" and args.sets == "causal" and args.layout == "bhnd":
         achieved = w["attn_flops"] / (res["attn_ms"] / 1e3) / 1e12
         line["roofline"] = {
             "kernel": "hybrid_chunk_attn_kernel", "bound": "tensor", "achieved": achieved, "peak": bf16_peak,
@@ -345,14 +349,14 @@ def run_ours(args):
                    "d2h_bytes_per_step": res["d2h"], "ms_per_step": res["e2e_ms"]}
     line["clocks"] = res["clocks"]
     line["gpu_launches"] = res["launches"]
-    if args.sets != "causal":  # one call per step: the path's fraction is the figure
+    if args.sets != "causal" or args.layout != "bhnd":  # one call per step: the path's fraction
         line["roofline"] = {"kernel": "whole path (states + fused attention)", "bound": "tensor",
                             "achieved": (w["attn_flops"] + w["state_flops"]) / (res["ms_step"] / 1e3) / 1e12,
                             "peak": bf16_peak, "unit": "TFLOP/s", "traffic": None,
                             "peak_source": f"{src} bf16 dense (burst)"}
         line["roofline"]["frac"] = line["roofline"]["achieved"] / bf16_peak
     if rank == 0 and world == 1 and not args.no_cpu_baseline and args.config == "wan13b" and not args.heads \
-            and args.sets == "causal":
+            and args.sets == "causal" and args.layout == "bhnd":
         rate, n, dt = oracle_sample_rate(c, res["q"], res["k"], res["v"], args.cpu_budget)
         line["cpu_baseline"] = {"value": rate, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
                                 "sample": f"fp64 explicit-mask oracle on {n} random query rows x all {c['H']} "
@@ -548,6 +552,7 @@ def main():
     ap.add_argument("--sweep", action="store_true")
     ap.add_argument("--compare-full", action="store_true", help="hybrid vs full softmax over (T_c, T_o)")
     ap.add_argument("--sets", choices=("causal", "bidirectional"), default="causal")
+    ap.add_argument("--layout", choices=("bhnd", "bnhd"), default="bhnd")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end leg (profiling runs)")
     ap.add_argument("--heads", type=int, default=0, help="override H (smaller profiling cases)")

@@ -114,7 +114,13 @@ int rehyat_forward_attention(const void* q, const void* k, const void* v,
 #define REHYAT_SETS_CAUSAL 0        /* §3.3 recurrent sets: T^L_t = { j < lo_t } (rehyat_forward) */
 #define REHYAT_SETS_BIDIRECTIONAL 1 /* §3.2 sets with overlap: T^L_t = T - T^S_t (earlier and later keys) */
 
-/* rehyat_forward with a choice of sets.  REHYAT_SETS_BIDIRECTIONAL is the
+/* Tensor layouts of rehyat_forward_ex (q, k, v and out share one). */
+#define REHYAT_LAYOUT_BHND 0  /* [B, H, N, d]: the layout of every other entry point */
+#define REHYAT_LAYOUT_BNHD 1  /* [B, N, H, d]: heads interleaved per token, as a DiT's
+                                 attention projection writes them (no transpose needed) */
+
+/* rehyat_forward with a choice of sets and of tensor layout.
+ * REHYAT_SETS_BIDIRECTIONAL is the
  * non-causal variant (§3.2 sets with overlap; the causal vs non-causal
  * comparison of §5.3): chunk t's linear term covers every key outside its
  * softmax window [lo_t, min((t+1)N', N)), later keys included, so it has no
@@ -126,7 +132,7 @@ int rehyat_forward_ex_workspace_bytes(int B, int H, int F, int S_tok, int d,
                                       size_t* bytes);
 int rehyat_forward_ex(const void* q, const void* k, const void* v,
                       int B, int H, int F, int S_tok, int d,
-                      int chunk_frames, int overlap_frames, int sets,
+                      int chunk_frames, int overlap_frames, int sets, int layout,
                       void* out, void* workspace, size_t workspace_bytes, void* stream);
 
 /* fp32 forward (SIMT fp32 throughout, accurate exp); same sets and layout.

@@ -12,20 +12,24 @@ namespace rehyat {
 // Fused per-chunk hybrid attention (tensor cores).  One CTA = one "unit":
 // up to two 128-row query tiles of one chunk of one (b,h).
 struct AttnParams {
-  CUtensorMap tm_q;   // [BH, N_q, D] bf16, box {64, 128, 1}, 128B swizzle
-  CUtensorMap tm_k;   // [BH, N_k, D]
-  CUtensorMap tm_v;   // [BH, N_k, D]
+  // q / k / v maps are 4-D {D, rows, H, B} with per-dimension strides (any of
+  // the [B,H,N,d] or [B,N,H,d] layouts), box {64, 128, 1, 1}, 128B swizzle.
+  CUtensorMap tm_q;
+  CUtensorMap tm_k;
+  CUtensorMap tm_v;
   CUtensorMap tm_hi;  // [BH * state_mul, 2D, D] bf16: high part of S_t
   CUtensorMap tm_lo;  // same: S_t - hi (rounded to bf16)
   ChunkGeom g;
   int BH;
+  int H;              // heads: bh = b * H + h
   int pairs;          // units per (bh, chunk)
   int state_mul;      // state tile z-coordinate = bh * state_mul + (g.step ? 0 : t)
   float scale_log2;   // log2(e) / sqrt(D)
   const float* z;     // z_t (fp32); entry e of (bh, t) at z[bh*z_bh + t*z_t + e]
   long long z_bh, z_t;
-  __nv_bfloat16* out; // [BH, N_q, D]
-  float* aS;          // diagnostic parts (PARTS kernels only)
+  __nv_bfloat16* out; // element (b, h, row, c) at out[b*o_sb + h*o_sh + row*o_sr + c]
+  long long o_sb, o_sh, o_sr;
+  float* aS;          // diagnostic parts, [BH, N_q, D] / [BH, N_q] (PARTS kernels only)
   float* nS;
   float* aL;
   float* nL;
@@ -36,10 +40,11 @@ struct AttnParams {
 // phi(K)^T V and sum phi(K) over key segments (tensor cores).  One CTA =
 // one piece of one segment of one (b,h).
 struct StateParams {
-  CUtensorMap tm_k;   // [BH, N_k, D] bf16, box {64, 64, 1}
+  CUtensorMap tm_k;   // 4-D {D, rows, H, B} bf16, box {64, 64, 1, 1}
   CUtensorMap tm_v;
   SegGeom sg;
   int BH;
+  int H;
   float* part_S;      // [BH, n_seg, nsplit, 2D, D] fp32
   float* part_z;      // [BH, n_seg, nsplit, 2D] fp32
 };

@@ -46,6 +46,8 @@ size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 struct FwdPlan {
   int BH, N, D, nc, n_seg, nsplit, chunk_tok, ovl_tok, pairs, n_units;
   int F, S_tok, tc, to, bidir;  // bidir: §3.2 sets (frame segments, prefix + suffix states)
+  int B, H;
+  long long rs, hs, bs;         // q/k/v/out element strides of a row, a head, a batch
   size_t off_pS, off_pz, off_hi, off_lo, off_zt, bytes;       // bf16 path
   size_t f32_off_pS, f32_off_pz, f32_off_S, f32_off_zt, f32_bytes;  // fp32 path
 };
@@ -62,6 +64,11 @@ int plan_forward(int B, int H, int F, int S_tok, int d, int Tc, int To, FwdPlan*
   const int tc = Tc < F ? Tc : F;
   const int to = To < F ? To : F;
   p->BH = static_cast<int>(BH);
+  p->B = B;
+  p->H = H;
+  p->rs = d;                      // [B, H, N, d] unless a layout says otherwise
+  p->hs = N * d;
+  p->bs = H * N * d;
   p->N = static_cast<int>(N);
   p->D = d;
   p->F = F;
@@ -132,7 +139,21 @@ int plan_forward_sets(int B, int H, int F, int S_tok, int d, int Tc, int To, int
   return REHYAT_OK;
 }
 
+// Element strides for a q/k/v/out layout.
+int apply_layout(int layout, FwdPlan* p) {
+  const long long N = p->N, d = p->D, H = p->H;
+  if (layout == REHYAT_LAYOUT_BHND) {
+    p->rs = d; p->hs = N * d; p->bs = H * N * d;
+  } else if (layout == REHYAT_LAYOUT_BNHD) {
+    p->rs = H * d; p->hs = d; p->bs = N * H * d;
+  } else {
+    return REHYAT_EINVAL;
+  }
+  return REHYAT_OK;
+}
+
 struct StepPlan {
+  int B, H;
   int BH, D, Nq, Nk, evict_tok, nsplit, pairs, n_units;
   size_t off_hi, off_lo, off_pS, off_pz, bytes;
   size_t f32_off_pS, f32_off_pz, f32_bytes;
@@ -149,6 +170,8 @@ int plan_step(int B, int H, int S_tok, int d, int qf, int cf, int ef, StepPlan* 
   if (BH > 65535 || Nk > INT_MAX / 2) return REHYAT_EINVAL;
   if (BH * Nk * d > (1LL << 46)) return REHYAT_EINVAL;
   p->BH = static_cast<int>(BH);
+  p->B = B;
+  p->H = H;
   p->D = d;
   p->Nq = static_cast<int>(Nq);
   p->Nk = static_cast<int>(Nk);
@@ -210,6 +233,24 @@ bool make_map(CUtensorMap* m, const void* base, long long inner, long long rows,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// bf16 tensor of B x H x rows x inner with arbitrary element strides for a
+// row, a head and a batch (inner is contiguous): 4-D map {inner, rows, H, B},
+// boxes of 64 x box_rows x 1 x 1, 128-byte swizzle, zero fill out of bounds.
+bool make_map4(CUtensorMap* m, const void* base, long long inner, long long rows, long long H, long long B,
+               long long rs, long long hs, long long bs, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[4] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(H),
+                        static_cast<cuuint64_t>(B)};
+  cuuint64_t strides[3] = {static_cast<cuuint64_t>(rs) * 2, static_cast<cuuint64_t>(hs) * 2,
+                           static_cast<cuuint64_t>(bs) * 2};
+  cuuint32_t box[4] = {64u, static_cast<cuuint32_t>(box_rows), 1u, 1u};
+  cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 int cuda_status(cudaError_t e) { return e == cudaSuccess ? REHYAT_OK : REHYAT_ECUDA; }
 
 #ifdef REHYAT_TRACE
@@ -226,10 +267,12 @@ int run_states(const void* k, const void* v, const FwdPlan& P, uint8_t* ws, floa
   if (P.n_seg > 0) {
     StateParams sp;
     std::memset(&sp, 0, sizeof(sp));
-    if (!make_map(&sp.tm_k, k, P.D, P.N, P.BH, 64) || !make_map(&sp.tm_v, v, P.D, P.N, P.BH, 64))
+    if (!make_map4(&sp.tm_k, k, P.D, P.N, P.H, P.B, P.rs, P.hs, P.bs, 64) ||
+        !make_map4(&sp.tm_v, v, P.D, P.N, P.H, P.B, P.rs, P.hs, P.bs, 64))
       return REHYAT_ECUDA;
     sp.sg = SegGeom{P.N, P.chunk_tok, P.ovl_tok, P.n_seg, P.nsplit, 0, 0, P.bidir ? P.S_tok : 0};
     sp.BH = P.BH;
+    sp.H = P.H;
     sp.part_S = pS;
     sp.part_z = pz;
     int st = cuda_status(launch_chunk_state(P.D, sp, P.BH * P.n_seg * P.nsplit, s));
@@ -259,13 +302,18 @@ int run_attention(const void* q, const void* k, const void* v, const FwdPlan& P,
                   float* aS, float* nS, float* aL, float* nL, float* Mo, cudaStream_t s) {
   AttnParams ap;
   std::memset(&ap, 0, sizeof(ap));
-  if (!make_map(&ap.tm_q, q, P.D, P.N, P.BH, 128) || !make_map(&ap.tm_k, k, P.D, P.N, P.BH, 128) ||
-      !make_map(&ap.tm_v, v, P.D, P.N, P.BH, 128) ||
+  if (!make_map4(&ap.tm_q, q, P.D, P.N, P.H, P.B, P.rs, P.hs, P.bs, 128) ||
+      !make_map4(&ap.tm_k, k, P.D, P.N, P.H, P.B, P.rs, P.hs, P.bs, 128) ||
+      !make_map4(&ap.tm_v, v, P.D, P.N, P.H, P.B, P.rs, P.hs, P.bs, 128) ||
       !make_map(&ap.tm_hi, ws + P.off_hi, P.D, 2LL * P.D, static_cast<long long>(P.BH) * P.nc, 128) ||
       !make_map(&ap.tm_lo, ws + P.off_lo, P.D, 2LL * P.D, static_cast<long long>(P.BH) * P.nc, 128))
     return REHYAT_ECUDA;
   ap.g = ChunkGeom{P.N, P.N, P.chunk_tok, P.ovl_tok, P.nc, 0};
   ap.BH = P.BH;
+  ap.H = P.H;
+  ap.o_sb = P.bs;
+  ap.o_sh = P.hs;
+  ap.o_sr = P.rs;
   ap.pairs = P.pairs;
   ap.state_mul = P.nc;
   ap.scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(P.D));
@@ -391,10 +439,12 @@ REHYAT_API int rehyat_forward_ex_workspace_bytes(int B, int H, int F, int S_tok,
 }
 
 REHYAT_API int rehyat_forward_ex(const void* q, const void* k, const void* v, int B, int H, int F, int S_tok, int d,
-                                 int chunk_frames, int overlap_frames, int sets, void* out, void* workspace,
-                                 size_t workspace_bytes, void* stream) {
+                                 int chunk_frames, int overlap_frames, int sets, int layout, void* out,
+                                 void* workspace, size_t workspace_bytes, void* stream) {
   FwdPlan P;
   int st = plan_forward_sets(B, H, F, S_tok, d, chunk_frames, overlap_frames, sets, &P);
+  if (st != REHYAT_OK) return st;
+  st = apply_layout(layout, &P);
   if (st != REHYAT_OK) return st;
   if (check_qkvo(q, k, v, out)) return REHYAT_EINVAL;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -519,12 +569,18 @@ REHYAT_API int rehyat_step_ws(const void* q_c, const void* k_c, const void* v_c,
   if (st != REHYAT_OK) return st;
   AttnParams ap;
   std::memset(&ap, 0, sizeof(ap));
-  if (!make_map(&ap.tm_q, q_c, P.D, P.Nq, P.BH, 128) || !make_map(&ap.tm_k, k_c, P.D, P.Nk, P.BH, 128) ||
-      !make_map(&ap.tm_v, v_c, P.D, P.Nk, P.BH, 128) || !make_map(&ap.tm_hi, hi, P.D, 2LL * P.D, P.BH, 128) ||
-      !make_map(&ap.tm_lo, lo, P.D, 2LL * P.D, P.BH, 128))
+  const long long d_ = P.D, H_ = P.H, Nq_ = P.Nq, Nk_ = P.Nk;
+  if (!make_map4(&ap.tm_q, q_c, P.D, P.Nq, P.H, P.B, d_, Nq_ * d_, H_ * Nq_ * d_, 128) ||
+      !make_map4(&ap.tm_k, k_c, P.D, P.Nk, P.H, P.B, d_, Nk_ * d_, H_ * Nk_ * d_, 128) ||
+      !make_map4(&ap.tm_v, v_c, P.D, P.Nk, P.H, P.B, d_, Nk_ * d_, H_ * Nk_ * d_, 128) ||
+      !make_map(&ap.tm_hi, hi, P.D, 2LL * P.D, P.BH, 128) || !make_map(&ap.tm_lo, lo, P.D, 2LL * P.D, P.BH, 128))
     return REHYAT_ECUDA;
   ap.g = ChunkGeom{P.Nq, P.Nk, P.Nq, 0, 1, 1};
   ap.BH = P.BH;
+  ap.H = P.H;
+  ap.o_sb = H_ * Nq_ * d_;
+  ap.o_sh = Nq_ * d_;
+  ap.o_sr = d_;
   ap.pairs = P.pairs;
   ap.state_mul = 1;
   ap.scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(P.D));
@@ -536,10 +592,12 @@ REHYAT_API int rehyat_step_ws(const void* q_c, const void* k_c, const void* v_c,
   if (st != REHYAT_OK || P.evict_tok == 0) return st;
   StateParams sp;
   std::memset(&sp, 0, sizeof(sp));
-  if (!make_map(&sp.tm_k, k_c, P.D, P.Nk, P.BH, 64) || !make_map(&sp.tm_v, v_c, P.D, P.Nk, P.BH, 64))
+  if (!make_map4(&sp.tm_k, k_c, P.D, P.Nk, P.H, P.B, d_, Nk_ * d_, H_ * Nk_ * d_, 64) ||
+      !make_map4(&sp.tm_v, v_c, P.D, P.Nk, P.H, P.B, d_, Nk_ * d_, H_ * Nk_ * d_, 64))
     return REHYAT_ECUDA;
   sp.sg = SegGeom{P.Nk, 0, 0, 1, P.nsplit, 1, P.evict_tok};
   sp.BH = P.BH;
+  sp.H = P.H;
   sp.part_S = reinterpret_cast<float*>(w + P.off_pS);
   sp.part_z = reinterpret_cast<float*>(w + P.off_pz);
   st = cuda_status(launch_chunk_state(P.D, sp, P.BH * P.nsplit, s));

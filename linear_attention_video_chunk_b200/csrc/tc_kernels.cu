@@ -338,7 +338,8 @@ __global__ void __launch_bounds__(384, 1) hybrid_chunk_attn_kernel(const __grid_
       if (ok) ok = warp_wait(BAR(C::B_O + X), 0, abort);
       tc_fence_after();
       const bool vrow = r < nX;
-      const size_t grow = static_cast<size_t>(bh) * p.g.N_q + (X ? rowB0 : rowA0) + r;
+      const int qrow = (X ? rowB0 : rowA0) + r;
+      const size_t grow = static_cast<size_t>(bh) * p.g.N_q + qrow;  // [BH, N_q] index (parts)
 
       if (PARTS && ok) {
 #pragma unroll
@@ -408,7 +409,8 @@ __global__ void __launch_bounds__(384, 1) hybrid_chunk_attn_kernel(const __grid_
             tmem_ld_wait();
             reg_fence(ov);
             if (vrow) {
-              uint4* dst = reinterpret_cast<uint4*>(p.out + grow * D + 32 * a);
+              uint4* dst = reinterpret_cast<uint4*>(p.out + (bh / p.H) * p.o_sb + (bh % p.H) * p.o_sh +
+                                                    qrow * p.o_sr + 32 * a);
 #pragma unroll
               for (int c = 0; c < 4; ++c) {
                 uint4 w;
@@ -449,25 +451,32 @@ __global__ void __launch_bounds__(384, 1) hybrid_chunk_attn_kernel(const __grid_
     if (lane == 0) {
       const uint32_t sq = smem_u32(smem + C::OFF_Q);
       const uint32_t ring = smem_u32(smem + C::OFF_RING);
+      const int hh = bh % p.H, bb = bh / p.H;
       mbar_arrive_expect_tx(BAR(C::B_Q), (hasB ? 2 : 1) * C::TILE_BYTES);
-      for (int b = 0; b < C::NBOX; ++b) tma_load_3d(sq + b * C::BOX_BYTES, &p.tm_q, BAR(C::B_Q), 64 * b, rowA0, bh);
+      for (int b = 0; b < C::NBOX; ++b) tma_load_4d(sq + b * C::BOX_BYTES, &p.tm_q, BAR(C::B_Q), 64 * b, rowA0, hh, bb);
       if (hasB)
         for (int b = 0; b < C::NBOX; ++b)
-          tma_load_3d(sq + C::TILE_BYTES + b * C::BOX_BYTES, &p.tm_q, BAR(C::B_Q), 64 * b, rowB0, bh);
+          tma_load_4d(sq + C::TILE_BYTES + b * C::BOX_BYTES, &p.tm_q, BAR(C::B_Q), 64 * b, rowB0, hh, bb);
       uint32_t seq = 0;
       bool ok = true;
+      // zc >= 0: a state tile (3-D map, depth zc); else a K/V tile (4-D map)
       auto load_tile = [&](const CUtensorMap* tm, int y, int zc) {
         const uint32_t slot = seq % NS;
         ok = ok && mbar_wait(BAR(C::B_EMPTY + slot), ((seq / NS) & 1) ^ 1, abort);
         if (!ok) return;
         mbar_arrive_expect_tx(BAR(C::B_FULL + slot), C::TILE_BYTES);
-        for (int b = 0; b < C::NBOX; ++b)
-          tma_load_3d(ring + slot * C::TILE_BYTES + b * C::BOX_BYTES, tm, BAR(C::B_FULL + slot), 64 * b, y, zc);
+        for (int b = 0; b < C::NBOX; ++b) {
+          const uint32_t dst = ring + slot * C::TILE_BYTES + b * C::BOX_BYTES;
+          if (zc >= 0)
+            tma_load_3d(dst, tm, BAR(C::B_FULL + slot), 64 * b, y, zc);
+          else
+            tma_load_4d(dst, tm, BAR(C::B_FULL + slot), 64 * b, y, hh, bb);
+        }
         ++seq;
       };
       for (int j = 0; j < ntiles && ok; ++j) {
-        load_tile(&p.tm_k, lo + 128 * j, bh);
-        load_tile(&p.tm_v, lo + 128 * j, bh);
+        load_tile(&p.tm_k, lo + 128 * j, -1);
+        load_tile(&p.tm_v, lo + 128 * j, -1);
       }
       if (has_lin) {
         const int zc = bh * p.state_mul + (p.g.step ? 0 : t);
@@ -791,8 +800,9 @@ __global__ void __launch_bounds__(StCfg<D>::THREADS, 1) phi_state_kernel(const _
         const uint32_t base = smem_u32(smem + st * C::STAGE);
         mbar_arrive_expect_tx(BAR(C::B_KV + st), 2 * C::KV_BYTES);
         for (int bb = 0; bb < C::NBOX; ++bb) {
-          tma_load_3d(base + bb * C::BOX, &p.tm_k, BAR(C::B_KV + st), 64 * bb, a + 64 * i, bh);
-          tma_load_3d(base + C::KV_BYTES + bb * C::BOX, &p.tm_v, BAR(C::B_KV + st), 64 * bb, a + 64 * i, bh);
+          tma_load_4d(base + bb * C::BOX, &p.tm_k, BAR(C::B_KV + st), 64 * bb, a + 64 * i, bh % p.H, bh / p.H);
+          tma_load_4d(base + C::KV_BYTES + bb * C::BOX, &p.tm_v, BAR(C::B_KV + st), 64 * bb, a + 64 * i, bh % p.H,
+                      bh / p.H);
         }
       }
       for (int i2 = (i > C::NST ? i - C::NST : 0); i2 < i; ++i2)

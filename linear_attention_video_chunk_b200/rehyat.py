@@ -38,12 +38,13 @@ _SIGS = {
     "rehyat_forward_noalloc": [_vp, _vp, _vp, _I, _I, _I, _I, _I, _I, _I, _vp, _vp],
     "rehyat_exp2_fma": [_vp, _vp, ctypes.c_int64, _vp],
     "rehyat_forward_ex_workspace_bytes": [_I, _I, _I, _I, _I, _I, _I, _I, ctypes.POINTER(_c_size)],
-    "rehyat_forward_ex": [_vp, _vp, _vp, _I, _I, _I, _I, _I, _I, _I, _I, _vp, _vp, _c_size, _vp],
+    "rehyat_forward_ex": [_vp, _vp, _vp, _I, _I, _I, _I, _I, _I, _I, _I, _I, _vp, _vp, _c_size, _vp],
 }
 _RESTYPES = {"rehyat_status_string": ctypes.c_char_p}
 
 OK, EINVAL, EUNSUPPORTED, ENOMEM, ECUDA, ETIMEOUT = range(6)
 SETS = {"causal": 0, "bidirectional": 1}
+LAYOUTS = {"bhnd": 0, "bnhd": 1}
 DTYPE_BF16, DTYPE_F32 = 0, 1
 
 _lib = None
@@ -137,19 +138,26 @@ def forward(q, k, v, F, S_tok, chunk_frames, overlap_frames, out=None, workspace
     return out
 
 
-def forward_sets(q, k, v, F, S_tok, chunk_frames, overlap_frames, sets="causal", out=None, workspace=None):
+def forward_sets(q, k, v, F, S_tok, chunk_frames, overlap_frames, sets="causal", layout="bhnd", out=None,
+                 workspace=None):
     """rehyat_forward_ex: the forward with the "causal" (§3.3, default) or
-    "bidirectional" (§3.2, non-causal) sets."""
+    "bidirectional" (§3.2, non-causal) sets, on [B,H,N,d] ("bhnd") or
+    [B,N,H,d] ("bnhd") tensors."""
     for n, t in (("q", q), ("k", k), ("v", v)):
         _need(t, torch.bfloat16, n)
-    B, H, N, d = _shape(q, F, S_tok)
+    if layout == "bhnd":
+        B, H, N, d = _shape(q, F, S_tok)
+    else:
+        B, N, H, d = q.shape
+        if N != F * S_tok:
+            raise ValueError(f"N={N} != F*S_tok={F * S_tok}")
     out = torch.empty_like(q) if out is None else out
     n = _c_size(0)
     _check(lib().rehyat_forward_ex_workspace_bytes(B, H, F, S_tok, d, chunk_frames, overlap_frames, SETS[sets],
                                                    ctypes.byref(n)), "rehyat_forward_ex_workspace_bytes")
     ws = alloc_workspace(n.value, q.device) if workspace is None else workspace
     _check(lib().rehyat_forward_ex(_p(q), _p(k), _p(v), B, H, F, S_tok, d, chunk_frames, overlap_frames, SETS[sets],
-                                   _p(out), _p(ws), ws.numel(), _stream()), "rehyat_forward_ex")
+                                   LAYOUTS[layout], _p(out), _p(ws), ws.numel(), _stream()), "rehyat_forward_ex")
     return out
 
 

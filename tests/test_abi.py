@@ -104,8 +104,10 @@ def test_ws_variants_check_workspace(lib):
 
 
 def test_forward_ex_validation(lib):
-    f = lambda sets, ws=0, nb=0: lib.rehyat_forward_ex(16, 16, 16, 1, 1, 4, 8, 64, 2, 1, sets, 16, ws, nb, None)
+    f = lambda sets, ws=0, nb=0, layout=0: lib.rehyat_forward_ex(16, 16, 16, 1, 1, 4, 8, 64, 2, 1, sets, layout,
+                                                                   16, ws, nb, None)
     assert f(2) == R.EINVAL              # unknown set mode
+    assert f(0, layout=2) == R.EINVAL    # unknown layout
     assert f(-1) == R.EINVAL
     assert f(1, ws=256, nb=1) == R.ENOMEM  # workspace too small (checked before launching)
     assert f(1, ws=272, nb=1 << 30) == R.EINVAL  # misaligned workspace

@@ -416,3 +416,28 @@ def test_wan13b_480p_bidirectional_sampled_rows():
     rows = few_rows(F, S, Tc)
     ref = orc.oracle_forward(q, k, v, F, S, Tc, To, mode="bidirectional", rows=rows)
     assert_bf16_close(np64(y[:, :, rows]), ref, "bidirectional 1.3B")
+
+
+# --------------------------------------------------------------------------- #
+# [B, N, H, d] layout                                                          #
+# --------------------------------------------------------------------------- #
+@pytest.mark.parametrize("sets", ["causal", "bidirectional"])
+@pytest.mark.parametrize("B,H,d,F,S,Tc,To,seed", [(2, 3, 128, 5, 200, 2, 1, 140), (1, 2, 64, 7, 90, 2, 3, 141)])
+def test_bnhd_layout_equals_bhnd_bitwise(sets, B, H, d, F, S, Tc, To, seed):
+    """Same arithmetic, different addressing: the [B,N,H,d] call on the
+    transposed tensors returns the transposed [B,H,N,d] result exactly."""
+    q, k, v = (x.cuda() for x in inputs.make_qkv(B, H, F * S, d, seed, rms_qk=True))
+    ref = R.forward_sets(q, k, v, F, S, Tc, To, sets=sets)
+    t = lambda x: x.transpose(1, 2).contiguous()
+    y = R.forward_sets(t(q), t(k), t(v), F, S, Tc, To, sets=sets, layout="bnhd")
+    assert torch.equal(y.transpose(1, 2), ref)
+
+
+def test_wan13b_480p_bnhd_sampled_rows():
+    B, H, d, F, S, Tc, To = 1, 12, 128, 21, 1560, 3, 1
+    q, k, v = inputs.make_qkv(B, H, F * S, d, 1, rms_qk=True)
+    t = lambda x: x.transpose(1, 2).contiguous().cuda()
+    y = R.forward_sets(t(q), t(k), t(v), F, S, Tc, To, layout="bnhd").transpose(1, 2).cpu()
+    rows = few_rows(F, S, Tc)
+    ref = orc.oracle_forward(q, k, v, F, S, Tc, To, rows=rows)
+    assert_bf16_close(np64(y[:, :, rows]), ref, "bnhd 1.3B")
