@@ -38,7 +38,7 @@ import math
 import numpy as np
 
 __all__ = [
-    "psi", "phi", "n_chunks", "chunk_geometry", "hybrid_mask_rows",
+    "psi", "phi", "phi_mlp", "mlp_identity_weights", "n_chunks", "chunk_geometry", "hybrid_mask_rows",
     "oracle_parts", "oracle_forward", "oracle_recurrent", "oracle_bruteforce",
     "oracle_chunk_states", "oracle_step",
 ]
@@ -67,6 +67,43 @@ def phi(x):
     """
     p = psi(x)
     return np.concatenate([p, p * p], axis=-1)
+
+
+def phi_mlp(x, W1, b1, W2, b2):
+    """Learned feature map ("ReHyAt", §4.3 Training specification and §7.1
+    Training Details): a two-layer MLP with degree-2 polynomial features,
+    phi(x) = [psi_1(x)^1, psi_2(x)^2] (the §3.2 feature-map equation, P = 2).
+    The pages fix neither the hidden width nor the output non-linearity; the
+    reading taken here is hidden width 2d and psi_p = 1 + elu of the MLP
+    outputs, which keeps phi non-negative (§3.1) and gives the paper's
+    parameter count.
+
+      h     = relu(W1 x + b1)             W1: [2d, d], b1: [2d]  (hidden 2d)
+      u     = W2 h + b2                   W2: [2d, 2d], b2: [2d]
+      psi_p = 1 + elu(u_p)                u_1 = u[:d], u_2 = u[d:]
+      phi   = [psi_1, psi_2 ** 2]         (non-negative, §3.1)
+
+    Per head and per map (q or k): 2d*d + 2d*2d = 98,304 weights at d = 128,
+    i.e. 2.36 M for the 12 heads of a block and both maps (the paper: about
+    2.4 M per converted block).  x: [..., d] -> [..., 2d] (float64).
+    """
+    x = np.asarray(x, dtype=np.float64)
+    d = x.shape[-1]
+    h = np.maximum(x @ np.asarray(W1, dtype=np.float64).T + np.asarray(b1, dtype=np.float64), 0.0)
+    u = h @ np.asarray(W2, dtype=np.float64).T + np.asarray(b2, dtype=np.float64)
+    p1 = psi(u[..., :d])
+    p2 = psi(u[..., d:])
+    return np.concatenate([p1, p2 * p2], axis=-1)
+
+
+def mlp_identity_weights(d):
+    """Weights with which phi_mlp is exactly the fixed map phi: the hidden
+    layer holds relu(x) and relu(-x) (W1 = [I; -I]) and each output block
+    recombines them to x (W2 rows [I, -I]), so u_1 = u_2 = x."""
+    I = np.eye(d)
+    W1 = np.concatenate([I, -I], axis=0)
+    W2 = np.concatenate([np.concatenate([I, -I], axis=1)] * 2, axis=0)
+    return W1, np.zeros(2 * d), W2, np.zeros(2 * d)
 
 
 # --------------------------------------------------------------------------- #
@@ -129,7 +166,7 @@ def _f64(x):
 # --------------------------------------------------------------------------- #
 # Parallel form, explicit mask                                                 #
 # --------------------------------------------------------------------------- #
-def oracle_parts(q, k, v, F, HW, T_c, T_o, mode="causal", rows=None, block=512):
+def oracle_parts(q, k, v, F, HW, T_c, T_o, mode="causal", rows=None, block=512, phi_q=None, phi_k=None):
     """The four unnormalised terms of the §3.2 joint normaliser, per query.
 
     For each (b, h) and query i of chunk t:
@@ -141,6 +178,8 @@ def oracle_parts(q, k, v, F, HW, T_c, T_o, mode="causal", rows=None, block=512):
     result raises.
 
     q, k, v: [B, H, N, d].  rows: optional query indices (all if None).
+    phi_q / phi_k: optional per-head feature maps, callables f(x, h) -> phi
+    (default: the fixed phi for both).
     Returns aS [B,H,R,d], nS [B,H,R], aL [B,H,R,d], nL [B,H,R] (float64).
     """
     q, k, v = _f64(q), _f64(k), _f64(v)
@@ -153,16 +192,18 @@ def oracle_parts(q, k, v, F, HW, T_c, T_o, mode="causal", rows=None, block=512):
     nS = np.zeros((B, H, R))
     nL = np.zeros((B, H, R))
     scale = 1.0 / math.sqrt(d)
+    fq = phi_q if phi_q is not None else (lambda x, h: phi(x))
+    fk = phi_k if phi_k is not None else (lambda x, h: phi(x))
     for b in range(B):
         for h in range(H):
             Q, K, V = q[b, h], k[b, h], v[b, h]
-            phiK = phi(K)
+            phiK = fk(K, h)
             for r0 in range(0, R, block):
                 rb = rows[r0:r0 + block]
                 in_S, in_L = hybrid_mask_rows(rb, F, HW, T_c, T_o, mode)
                 s = (Q[rb] @ K.T) * scale
                 wS = np.exp(np.where(in_S, s, -np.inf))
-                wL = np.where(in_L, phi(Q[rb]) @ phiK.T, 0.0)
+                wL = np.where(in_L, fq(Q[rb], h) @ phiK.T, 0.0)
                 aS[b, h, r0:r0 + rb.size] = wS @ V
                 nS[b, h, r0:r0 + rb.size] = wS.sum(axis=1)
                 aL[b, h, r0:r0 + rb.size] = wL @ V
@@ -172,10 +213,10 @@ def oracle_parts(q, k, v, F, HW, T_c, T_o, mode="causal", rows=None, block=512):
     return aS, nS, aL, nL
 
 
-def oracle_forward(q, k, v, F, HW, T_c, T_o, mode="causal", rows=None, block=512):
+def oracle_forward(q, k, v, F, HW, T_c, T_o, mode="causal", rows=None, block=512, phi_q=None, phi_k=None):
     """Hybrid attention output y_i = (a^S + a^L) / (n^S + n^L)  (§3.2 joint
     normalisation), with the sets of ``mode``.  Returns [B, H, R, d] float64."""
-    aS, nS, aL, nL = oracle_parts(q, k, v, F, HW, T_c, T_o, mode, rows, block)
+    aS, nS, aL, nL = oracle_parts(q, k, v, F, HW, T_c, T_o, mode, rows, block, phi_q, phi_k)
     return (aS + aL) / (nS + nL)[..., None]
 
 
@@ -202,7 +243,7 @@ def oracle_chunk_states(k, v, F, HW, T_c, T_o):
     return S, z
 
 
-def oracle_recurrent(q, k, v, F, HW, T_c, T_o):
+def oracle_recurrent(q, k, v, F, HW, T_c, T_o, phi_q=None, phi_k=None):
     """§3.3 chunk-wise RNN: walk the chunks in order with a constant-size state.
 
     Before chunk t the state (S, z) is advanced by folding in the keys
@@ -215,6 +256,8 @@ def oracle_recurrent(q, k, v, F, HW, T_c, T_o):
     B, H, N, d = q.shape
     out = np.zeros_like(q)
     scale = 1.0 / math.sqrt(d)
+    fq = phi_q if phi_q is not None else (lambda x, h: phi(x))
+    fk = phi_k if phi_k is not None else (lambda x, h: phi(x))
     for b in range(B):
         for h in range(H):
             Q, K, V = q[b, h], k[b, h], v[b, h]
@@ -223,12 +266,12 @@ def oracle_recurrent(q, k, v, F, HW, T_c, T_o):
             folded = 0
             for t in range(n_chunks(F, T_c)):
                 q0, q1, lo, hi = chunk_geometry(t, F, HW, T_c, T_o)
-                pk = phi(K[folded:lo])
+                pk = fk(K[folded:lo], h)
                 S = S + pk.T @ V[folded:lo]
                 z = z + pk.sum(axis=0)
                 folded = lo
                 e = np.exp((Q[q0:q1] @ K[lo:hi].T) * scale)
-                pq = phi(Q[q0:q1])
+                pq = fq(Q[q0:q1], h)
                 num = e @ V[lo:hi] + pq @ S
                 den = e.sum(axis=1) + pq @ z
                 out[b, h, q0:q1] = num / den[:, None]
@@ -263,10 +306,14 @@ def oracle_step(q_c, k_c, v_c, S, z, HW, evict_frames):
 # --------------------------------------------------------------------------- #
 # Brute force (pure Python, tiny inputs only)                                  #
 # --------------------------------------------------------------------------- #
-def oracle_bruteforce(q, k, v, F, HW, T_c, T_o, mode="causal"):
+def oracle_bruteforce(q, k, v, F, HW, T_c, T_o, mode="causal", phi_q=None, phi_k=None):
     """Double loop over (query, key) pairs with set membership decided inline
     from the §3.2 / §3.3 set definitions: no mask matrix, no numpy algebra.
-    Intended for N <= ~64 and d <= ~8.  Returns nested lists [B][H][N][d]."""
+    Intended for N <= ~64 and d <= ~8.  Returns nested lists [B][H][N][d].
+
+    phi_q / phi_k: optional per-vector feature maps f(x, h) -> sequence of
+    D' floats; the linear weight is then their dot product, summed in a loop
+    (default: the fixed phi, inline per element)."""
     q, k, v = _f64(q), _f64(k), _f64(v)
     B, H, N, d = q.shape
     Np = T_c * HW
@@ -299,6 +346,12 @@ def oracle_bruteforce(q, k, v, F, HW, T_c, T_o, mode="causal"):
                         for c in range(d):
                             dot += q[b, h, i, c] * k[b, h, j, c]
                         w = math.exp(dot * rs)
+                    elif glob and phi_q is not None:
+                        fa = list(phi_q(q[b, h, i], h))
+                        fb = list(phi_k(k[b, h, j], h))
+                        w = 0.0
+                        for e in range(len(fa)):
+                            w += fa[e] * fb[e]
                     elif glob:
                         w = 0.0
                         for c in range(d):

@@ -328,10 +328,10 @@ def test_planted_scale_mistake_is_caught(monkeypatch):
     carry 1/d and phi sees scaled queries)."""
     orig_parts = orc.oracle_parts
 
-    def parts(q, k, v, F, HW, T_c, T_o, mode="causal", rows=None, block=512):
+    def parts(q, k, v, F, HW, T_c, T_o, mode="causal", rows=None, block=512, phi_q=None, phi_k=None):
         d = np.asarray(q).shape[-1]
         s = 1.0 / math.sqrt(d)
-        return orig_parts(np.asarray(q) * s, k, v, F, HW, T_c, T_o, mode, rows, block)
+        return orig_parts(np.asarray(q) * s, k, v, F, HW, T_c, T_o, mode, rows, block, phi_q, phi_k)
     monkeypatch.setattr(orc, "oracle_parts", parts)
     assert not _pins_hold()
 
@@ -340,7 +340,163 @@ def test_planted_transposed_kv_is_caught(monkeypatch):
     """Keys and values swapped inside the parallel oracle."""
     orig_parts = orc.oracle_parts
 
-    def parts(q, k, v, F, HW, T_c, T_o, mode="causal", rows=None, block=512):
-        return orig_parts(q, v, k, F, HW, T_c, T_o, mode, rows, block)
+    def parts(q, k, v, F, HW, T_c, T_o, mode="causal", rows=None, block=512, phi_q=None, phi_k=None):
+        return orig_parts(q, v, k, F, HW, T_c, T_o, mode, rows, block, phi_q, phi_k)
     monkeypatch.setattr(orc, "oracle_parts", parts)
     assert not _pins_hold()
+
+
+# --------------------------------------------------------------------------- #
+# learned feature map: two-layer MLP with degree-2 polynomial features         #
+# --------------------------------------------------------------------------- #
+def _mlp_weights(H, d, seed, scale=1.0):
+    """Random (non-symmetric) per-head weights, W1 [H,2d,d], W2 [H,2d,2d]."""
+    g = np.random.default_rng(seed)
+    return (g.standard_normal((H, 2 * d, d)) * scale / math.sqrt(d), g.standard_normal((H, 2 * d)) * 0.3,
+            g.standard_normal((H, 2 * d, 2 * d)) * scale / math.sqrt(2 * d), g.standard_normal((H, 2 * d)) * 0.3)
+
+
+def _maps(Wq, Wk):
+    fq = lambda x, h: orc.phi_mlp(x, Wq[0][h], Wq[1][h], Wq[2][h], Wq[3][h])
+    fk = lambda x, h: orc.phi_mlp(x, Wk[0][h], Wk[1][h], Wk[2][h], Wk[3][h])
+    return fq, fk
+
+
+@pytest.mark.parametrize("d", [3, 8])
+def test_phi_mlp_matches_torch_modules(d):
+    """phi_mlp == torch.nn.Linear -> ReLU -> Linear, then 1 + torch elu on
+    each output half and the square of the second (P = 2 of the §3.2
+    feature-map equation), in fp64 with the same weights."""
+    W1, b1, W2, b2 = (w[0] for w in _mlp_weights(1, d, 5 + d))
+    x = _rand((13, d), 7 + d, 2.0)
+    l1 = torch.nn.Linear(d, 2 * d).double()
+    l2 = torch.nn.Linear(2 * d, 2 * d).double()
+    with torch.no_grad():
+        l1.weight.copy_(torch.from_numpy(W1))
+        l1.bias.copy_(torch.from_numpy(b1))
+        l2.weight.copy_(torch.from_numpy(W2))
+        l2.bias.copy_(torch.from_numpy(b2))
+        u = l2(torch.relu(l1(torch.from_numpy(x))))
+        p1 = 1.0 + torch.nn.functional.elu(u[:, :d])
+        p2 = 1.0 + torch.nn.functional.elu(u[:, d:])
+        want = torch.cat([p1, p2 ** 2], dim=1).numpy()
+    got = orc.phi_mlp(x, W1, b1, W2, b2)
+    np.testing.assert_allclose(got, want, rtol=1e-14, atol=1e-14)
+    assert (got >= 0).all()
+
+
+def test_phi_mlp_identity_weights_reduce_to_fixed_phi():
+    """With W1 = [I; -I], W2 rows [I, -I] and zero biases the MLP outputs
+    u = x, so the learned map is exactly the fixed phi, and the forward with
+    those maps is the fixed-phi forward."""
+    d = 6
+    x = _rand((40, d), 11, 3.0)
+    np.testing.assert_array_equal(orc.phi_mlp(x, *orc.mlp_identity_weights(d)), orc.phi(x))
+    q, k, v = _qkv(1, 2, 20, d, 13)
+    f = lambda x, h: orc.phi_mlp(x, *orc.mlp_identity_weights(d))
+    np.testing.assert_allclose(orc.oracle_forward(q, k, v, 5, 4, 2, 1, phi_q=f, phi_k=f),
+                               orc.oracle_forward(q, k, v, 5, 4, 2, 1), rtol=1e-13, atol=1e-14)
+
+
+@pytest.mark.parametrize("F,HW,Tc,To", [(5, 4, 2, 1), (6, 3, 1, 2)])
+def test_constant_features_closed_form(F, HW, Tc, To):
+    """W2 = 0: every token gets the same features c = [psi(b2_1), psi(b2_2)^2].
+    Linear-only attention is then the plain mean of V; in the causal sets every
+    linear key weighs |c|^2, so y_i = (sum_S e^s v + |c|^2 sum_L v) /
+    (sum_S e^s + |c|^2 |L|) with the sets counted from the §3.3 definitions."""
+    d, N = 4, F * HW
+    q, k, v = _qkv(1, 1, N, d, 17)
+    W1, b1, W2, b2 = (w[0] for w in _mlp_weights(1, d, 19))
+    W2 = np.zeros_like(W2)
+    f = lambda x, h: orc.phi_mlp(x, W1, b1, W2, b2)
+    lin = orc.oracle_forward(q, k, v, F, HW, Tc, To, mode="linear_only", phi_q=f, phi_k=f)
+    np.testing.assert_allclose(lin[0, 0], np.broadcast_to(v[0, 0].mean(axis=0), (N, d)), rtol=1e-12)
+    c = np.concatenate([orc.psi(b2[:d]), orc.psi(b2[d:]) ** 2])
+    w = float(c @ c)
+    got = orc.oracle_forward(q, k, v, F, HW, Tc, To, phi_q=f, phi_k=f)[0, 0]
+    Np = Tc * HW
+    for i in range(N):
+        t = i // Np
+        lo, hi = max(t * Np - To * HW, 0), min((t + 1) * Np, N)
+        e = np.exp(k[0, 0, lo:hi] @ q[0, 0, i] / math.sqrt(d))
+        num = e @ v[0, 0, lo:hi] + w * v[0, 0, :lo].sum(axis=0)
+        den = e.sum() + w * lo
+        np.testing.assert_allclose(got[i], num / den, rtol=1e-12)
+
+
+@pytest.mark.parametrize("F,HW,Tc,To", [(7, 5, 3, 1), (6, 4, 2, 3), (5, 3, 1, 0)])
+def test_mlp_recurrent_equals_parallel(F, HW, Tc, To):
+    """§3.3 RNN form == explicit-mask parallel form with separate learned
+    phi_q and phi_k per head."""
+    d, H = 5, 2
+    q, k, v = _qkv(1, H, F * HW, d, 23)
+    fq, fk = _maps(_mlp_weights(H, d, 29), _mlp_weights(H, d, 31))
+    par = orc.oracle_forward(q, k, v, F, HW, Tc, To, phi_q=fq, phi_k=fk)
+    rec = orc.oracle_recurrent(q, k, v, F, HW, Tc, To, phi_q=fq, phi_k=fk)
+    np.testing.assert_allclose(rec, par, rtol=1e-12, atol=1e-13)
+
+
+@pytest.mark.parametrize("mode", ["causal", "bidirectional", "linear_only"])
+def test_mlp_bruteforce_equals_mask_oracle(mode):
+    """Scalar loops with per-pair feature dot products == mask oracle, with
+    phi_q != phi_k (a swap of the two maps changes the result)."""
+    F, HW, Tc, To, d, H = 4, 3, 2, 1, 3, 2
+    q, k, v = _qkv(1, H, F * HW, d, 37)
+    fq, fk = _maps(_mlp_weights(H, d, 41), _mlp_weights(H, d, 43))
+    got = orc.oracle_forward(q, k, v, F, HW, Tc, To, mode=mode, phi_q=fq, phi_k=fk)
+    bf = np.array(orc.oracle_bruteforce(q, k, v, F, HW, Tc, To, mode=mode, phi_q=fq, phi_k=fk))
+    np.testing.assert_allclose(got, bf, rtol=1e-12, atol=1e-13)
+    swapped = orc.oracle_forward(q, k, v, F, HW, Tc, To, mode=mode, phi_q=fk, phi_k=fq)
+    assert np.abs(swapped - bf).max() > 1e-6
+
+
+def _mlp_pins_hold():
+    try:
+        test_phi_mlp_matches_torch_modules(3)
+        test_constant_features_closed_form(5, 4, 2, 1)
+        test_mlp_bruteforce_equals_mask_oracle("causal")
+    except AssertionError:
+        return False
+    return True
+
+
+def test_unmodified_mlp_oracle_passes_pins():
+    assert _mlp_pins_hold()
+
+
+def _mlp_mutant(kind):
+    orig = orc.phi_mlp
+
+    def m(x, W1, b1, W2, b2):
+        W1, W2 = np.asarray(W1), np.asarray(W2)
+        if kind == "no_hidden_bias":
+            return orig(x, W1, np.zeros_like(b1), W2, b2)
+        if kind == "transposed_w2":
+            return orig(x, W1, b1, W2.T, b2)
+        if kind == "no_relu":
+            x = np.asarray(x, dtype=np.float64)
+            d = x.shape[-1]
+            u = (x @ W1.T + b1) @ W2.T + b2
+            return np.concatenate([orc.psi(u[..., :d]), orc.psi(u[..., d:]) ** 2], -1)
+        if kind == "no_square":
+            y = orig(x, W1, b1, W2, b2)
+            d = y.shape[-1] // 2
+            return np.concatenate([y[..., :d], np.sqrt(y[..., d:])], -1)
+        raise ValueError(kind)
+    return m
+
+
+@pytest.mark.parametrize("kind", ["no_hidden_bias", "transposed_w2", "no_relu", "no_square"])
+def test_planted_mlp_mistake_is_caught(kind, monkeypatch):
+    monkeypatch.setattr(orc, "phi_mlp", _mlp_mutant(kind))
+    assert not _mlp_pins_hold(), f"planted mistake {kind} went unnoticed"
+
+
+def test_planted_swapped_maps_is_caught(monkeypatch):
+    """phi_q and phi_k exchanged inside the parallel oracle."""
+    orig_parts = orc.oracle_parts
+
+    def parts(q, k, v, F, HW, T_c, T_o, mode="causal", rows=None, block=512, phi_q=None, phi_k=None):
+        return orig_parts(q, k, v, F, HW, T_c, T_o, mode, rows, block, phi_k, phi_q)
+    monkeypatch.setattr(orc, "oracle_parts", parts)
+    assert not _mlp_pins_hold()
