@@ -163,6 +163,14 @@ def _f64(x):
     return np.asarray(x, dtype=np.float64)
 
 
+def _features(f, X, idx, b, h):
+    """phi of the rows idx of X (one head): f is a per-head map f(x, h), or an
+    array [B, H, N, D'] of precomputed features indexed by (b, h, row)."""
+    if callable(f):
+        return f(X[idx], h)
+    return np.asarray(f, dtype=np.float64)[b, h][idx]
+
+
 # --------------------------------------------------------------------------- #
 # Parallel form, explicit mask                                                 #
 # --------------------------------------------------------------------------- #
@@ -178,8 +186,8 @@ def oracle_parts(q, k, v, F, HW, T_c, T_o, mode="causal", rows=None, block=512, 
     result raises.
 
     q, k, v: [B, H, N, d].  rows: optional query indices (all if None).
-    phi_q / phi_k: optional per-head feature maps, callables f(x, h) -> phi
-    (default: the fixed phi for both).
+    phi_q / phi_k: optional per-head feature maps, callables f(x, h) -> phi,
+    or arrays [B, H, N, D'] of precomputed features (default: the fixed phi).
     Returns aS [B,H,R,d], nS [B,H,R], aL [B,H,R,d], nL [B,H,R] (float64).
     """
     q, k, v = _f64(q), _f64(k), _f64(v)
@@ -197,13 +205,13 @@ def oracle_parts(q, k, v, F, HW, T_c, T_o, mode="causal", rows=None, block=512, 
     for b in range(B):
         for h in range(H):
             Q, K, V = q[b, h], k[b, h], v[b, h]
-            phiK = fk(K, h)
+            phiK = _features(fk, K, slice(None), b, h)
             for r0 in range(0, R, block):
                 rb = rows[r0:r0 + block]
                 in_S, in_L = hybrid_mask_rows(rb, F, HW, T_c, T_o, mode)
                 s = (Q[rb] @ K.T) * scale
                 wS = np.exp(np.where(in_S, s, -np.inf))
-                wL = np.where(in_L, fq(Q[rb], h) @ phiK.T, 0.0)
+                wL = np.where(in_L, _features(fq, Q, rb, b, h) @ phiK.T, 0.0)
                 aS[b, h, r0:r0 + rb.size] = wS @ V
                 nS[b, h, r0:r0 + rb.size] = wS.sum(axis=1)
                 aL[b, h, r0:r0 + rb.size] = wL @ V
@@ -266,12 +274,12 @@ def oracle_recurrent(q, k, v, F, HW, T_c, T_o, phi_q=None, phi_k=None):
             folded = 0
             for t in range(n_chunks(F, T_c)):
                 q0, q1, lo, hi = chunk_geometry(t, F, HW, T_c, T_o)
-                pk = fk(K[folded:lo], h)
+                pk = _features(fk, K, slice(folded, lo), b, h)
                 S = S + pk.T @ V[folded:lo]
                 z = z + pk.sum(axis=0)
                 folded = lo
                 e = np.exp((Q[q0:q1] @ K[lo:hi].T) * scale)
-                pq = fq(Q[q0:q1], h)
+                pq = _features(fq, Q, slice(q0, q1), b, h)
                 num = e @ V[lo:hi] + pq @ S
                 den = e.sum(axis=1) + pq @ z
                 out[b, h, q0:q1] = num / den[:, None]

@@ -450,6 +450,21 @@ def test_mlp_bruteforce_equals_mask_oracle(mode):
     assert np.abs(swapped - bf).max() > 1e-6
 
 
+def test_precomputed_feature_arrays_equal_maps():
+    """Feature arrays [B,H,N,D'] stand in for the maps that produced them, in
+    the parallel and the recurrent form."""
+    F, HW, Tc, To, d, H = 5, 4, 2, 1, 4, 2
+    q, k, v = _qkv(2, H, F * HW, d, 47)
+    fq, fk = _maps(_mlp_weights(H, d, 53), _mlp_weights(H, d, 59))
+    Pq = np.stack([np.stack([fq(q[b, h], h) for h in range(H)]) for b in range(2)])
+    Pk = np.stack([np.stack([fk(k[b, h], h) for h in range(H)]) for b in range(2)])
+    want = orc.oracle_forward(q, k, v, F, HW, Tc, To, phi_q=fq, phi_k=fk)
+    np.testing.assert_allclose(orc.oracle_forward(q, k, v, F, HW, Tc, To, phi_q=Pq, phi_k=Pk, block=7), want,
+                               rtol=1e-13, atol=1e-14)
+    np.testing.assert_allclose(orc.oracle_recurrent(q, k, v, F, HW, Tc, To, phi_q=Pq, phi_k=Pk), want,
+                               rtol=1e-12, atol=1e-13)
+
+
 def _mlp_pins_hold():
     try:
         test_phi_mlp_matches_torch_modules(3)
