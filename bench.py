@@ -68,8 +68,11 @@ def work(c, sets="causal"):
     state_flops = BH * 2 * D2 * (d + 1) * folded
     attn_bytes = BH * N * d * 2 * 4 + BH * len(ch) * D2 * (d * 4 + 4)     # q,k,v,out + states (hi,lo,z)
     state_bytes = BH * folded * d * 2 * 2 + BH * len(ch) * D2 * (d * 4 + 4)
+    # learned feature map, both maps: x [N, d] -> relu(W1 x) [N, 2d] -> phi [N, 2d]
+    mlp_flops = 2 * BH * N * 2 * (D2 * d + D2 * D2)
+    mlp_bytes = 2 * (BH * N * (d + D2) * 2 + H * (D2 * d + D2 * D2) * 2 + H * 2 * D2 * 4)
     return dict(pairs_per_head=pairs, attn_flops=attn_flops, state_flops=state_flops, attn_bytes=attn_bytes,
-                state_bytes=state_bytes, tokens=B * N)
+                state_bytes=state_bytes, tokens=B * N, mlp_flops=mlp_flops, mlp_bytes=mlp_bytes)
 
 
 KERNEL_SOURCES = ("tc_kernels.cu", "ptx.cuh", "kernels.cuh", "geom.cuh")
@@ -218,7 +221,13 @@ def run_forward_bench(args, c, rank, world, dev):
     ws = R.alloc_workspace(R.workspace_bytes(B, H, F, S, d, Tc, To), dev)
     torch.cuda.synchronize()
 
-    if args.sets != "causal" or args.layout != "bhnd":  # one call (states + attention) per step
+    mlp = args.phi == "mlp"
+    one_call = args.sets != "causal" or args.layout != "bhnd" or mlp
+    if mlp:  # learned feature maps: resident weights, phi(q) and phi(k) computed every step
+        wq = tuple(t.to(dev) for t in inputs.make_mlp_weights(H, d, c["seed"], "q"))
+        wk = tuple(t.to(dev) for t in inputs.make_mlp_weights(H, d, c["seed"], "k"))
+        ws = R.alloc_workspace(R.forward_mlp_workspace_bytes(B, H, F, S, d, Tc, To, args.sets), dev)
+    elif one_call:  # one call (states + attention) per step
         n = R.ctypes.c_size_t(0)
         R.lib().rehyat_forward_ex_workspace_bytes(B, H, F, S, d, Tc, To, R.SETS[args.sets], R.ctypes.byref(n))
         ws = R.alloc_workspace(n.value, dev)
@@ -226,7 +235,12 @@ def run_forward_bench(args, c, rank, world, dev):
     def step(e0=None, e1=None, e2=None):
         if e0 is not None:
             e0.record()
-        if args.sets != "causal" or args.layout != "bhnd":
+        if mlp:
+            if e1 is not None:
+                e1.record()
+            R.forward_mlp(qd, kd, vd, wq, wk, F, S, Tc, To, sets=args.sets, layout=args.layout, out=out,
+                          workspace=ws)
+        elif one_call:
             if e1 is not None:
                 e1.record()
             R.forward_sets(qd, kd, vd, F, S, Tc, To, sets=args.sets, layout=args.layout, out=out, workspace=ws)
@@ -257,17 +271,36 @@ def run_forward_bench(args, c, rank, world, dev):
     ms_step = max_over_ranks(start.elapsed_time(end) / K, world, dev)
     attn_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in ev)
     state_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
+    mlp_ms = None
+    if mlp:  # the feature-map kernel alone (one map per launch), for its roofline
+        phi_out = torch.empty((B, H, N, 2 * d), dtype=torch.bfloat16, device=dev)
+        src = qd
+        for _ in range(3):
+            R.phi_mlp(src, *wq, layout=args.layout, out=phi_out)
+        m0, m1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        Km = max(3, min(K, 50))
+        m0.record()
+        for _ in range(Km):
+            R.phi_mlp(src, *wq, layout=args.layout, out=phi_out)
+        m1.record()
+        torch.cuda.synchronize()
+        mlp_ms = m0.elapsed_time(m1) / Km
+        del phi_out
 
     # end to end through the public API: pinned host inputs -> device ->
     # forward -> result back to pinned host memory, every step
+    launches = (4 if mlp else 3) * K
     if args.no_e2e:
         return dict(ms_step=ms_step, attn_ms=attn_ms, state_ms=state_ms, e2e_ms=float("nan"), clocks=clk.summary(),
-                    h2d=0, d2h=0, q=q, k=k, v=v, launches=3 * K)
+                    h2d=0, d2h=0, q=q, k=k, v=v, launches=launches, mlp_ms=mlp_ms)
     out_h = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
     Ke = max(3, min(K, 20))
 
     def fwd(o):  # the public API call a user makes
-        if args.sets == "causal" and args.layout == "bhnd":
+        if mlp:
+            R.forward_mlp(qd, kd, vd, wq, wk, F, S, Tc, To, sets=args.sets, layout=args.layout, out=o,
+                          workspace=ws)
+        elif args.sets == "causal" and args.layout == "bhnd":
             R.forward(qd, kd, vd, F, S, Tc, To, out=o, workspace=ws)
         else:
             R.forward_sets(qd, kd, vd, F, S, Tc, To, sets=args.sets, layout=args.layout, out=o, workspace=ws)
@@ -295,7 +328,7 @@ def run_forward_bench(args, c, rank, world, dev):
         raise RuntimeError(f"device status {R.status_string(status)}")
     return dict(ms_step=ms_step, attn_ms=attn_ms, state_ms=state_ms, e2e_ms=e2e_ms, clocks=clk.summary(),
                 h2d=3 * q.numel() * q.element_size(), d2h=out.numel() * out.element_size(), q=q, k=k, v=v,
-                launches=3 * K)
+                launches=launches, mlp_ms=mlp_ms)
 
 
 def run_ours(args):
@@ -314,6 +347,8 @@ def run_ours(args):
         c["H"] = args.heads
         c["workload"] += f" (H overridden to {args.heads})"
     if args.config == "recurrent":
+        if args.phi != "fixed":
+            raise SystemExit("--phi mlp is measured on the parallel form (wan13b, wan14b)")
         res = run_recurrent_bench(args, c, rank, world, dev)
     else:
         res = run_forward_bench(args, c, rank, world, dev)
@@ -324,6 +359,8 @@ def run_ours(args):
         c["workload"] += f" ({args.sets} sets)"
     if args.layout != "bhnd":
         c["workload"] += " ([B, N, H, d] layout)"
+    if args.phi == "mlp":
+        c["workload"] += " (learned phi: 2-layer MLP, degree-2 features)"
     line = {
         "metric": METRIC, "value": tokens / (res["ms_step"] / 1e3), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": res["ms_step"], "higher_is_better": True,
@@ -334,7 +371,7 @@ def run_ours(args):
                    "tokens_per_step_per_gpu": w["tokens"], "parallelism": f"replicas x{world} (no collective)",
                    "l2": "inputs larger than L2: q+k+v = %.0f MB per GPU" % (3 * w["tokens"] * c["H"] * c["d"] * 2 / 1e6)},
     }
-    if args.config != "recurrent" and args.sets == "causal" and args.layout == "bhnd":
+    if args.config != "recurrent" and args.sets == "causal" and args.layout == "bhnd" and args.phi == "fixed":
         achieved = w["attn_flops"] / (res["attn_ms"] / 1e3) / 1e12
         line["roofline"] = {
             "kernel": "hybrid_chunk_attn_kernel", "bound": "tensor", "achieved": achieved, "peak": bf16_peak,
@@ -349,14 +386,24 @@ def run_ours(args):
                    "d2h_bytes_per_step": res["d2h"], "ms_per_step": res["e2e_ms"]}
     line["clocks"] = res["clocks"]
     line["gpu_launches"] = res["launches"]
-    if args.sets != "causal" or args.layout != "bhnd":  # one call per step: the path's fraction
-        line["roofline"] = {"kernel": "whole path (states + fused attention)", "bound": "tensor",
-                            "achieved": (w["attn_flops"] + w["state_flops"]) / (res["ms_step"] / 1e3) / 1e12,
+    if args.config != "recurrent" and (args.sets != "causal" or args.layout != "bhnd" or args.phi == "mlp"):
+        # one call per step: the whole path's fraction
+        flops = w["attn_flops"] + w["state_flops"] + (w["mlp_flops"] if args.phi == "mlp" else 0)
+        line["roofline"] = {"kernel": "whole path (%sstates + fused attention)" %
+                                      ("phi MLP + " if args.phi == "mlp" else ""), "bound": "tensor",
+                            "achieved": flops / (res["ms_step"] / 1e3) / 1e12,
                             "peak": bf16_peak, "unit": "TFLOP/s", "traffic": None,
                             "peak_source": f"{src} bf16 dense (burst)"}
         line["roofline"]["frac"] = line["roofline"]["achieved"] / bf16_peak
+    if res.get("mlp_ms"):
+        t = res["mlp_ms"] / 1e3
+        fl = w["mlp_flops"] / 2 / t / 1e12       # one map per timed launch
+        gbs = w["mlp_bytes"] / 2 / t / 1e9
+        line["phi_mlp_kernel"] = {"kernel": "phi_mlp_kernel (one map)", "ms": res["mlp_ms"],
+                                  "tflops": fl, "frac_tensor": fl / bf16_peak, "gbs": gbs, "frac_hbm": gbs / hbm,
+                                  "flops_per_launch": w["mlp_flops"] // 2, "bytes_per_launch": w["mlp_bytes"] // 2}
     if rank == 0 and world == 1 and not args.no_cpu_baseline and args.config == "wan13b" and not args.heads \
-            and args.sets == "causal" and args.layout == "bhnd":
+            and args.sets == "causal" and args.layout == "bhnd" and args.phi == "fixed":
         rate, n, dt = oracle_sample_rate(c, res["q"], res["k"], res["v"], args.cpu_budget)
         line["cpu_baseline"] = {"value": rate, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
                                 "sample": f"fp64 explicit-mask oracle on {n} random query rows x all {c['H']} "
@@ -553,6 +600,8 @@ def main():
     ap.add_argument("--compare-full", action="store_true", help="hybrid vs full softmax over (T_c, T_o)")
     ap.add_argument("--sets", choices=("causal", "bidirectional"), default="causal")
     ap.add_argument("--layout", choices=("bhnd", "bnhd"), default="bhnd")
+    ap.add_argument("--phi", choices=("fixed", "mlp"), default="fixed",
+                    help="feature map: fixed 1+elu features, or the learned two-layer MLP")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end leg (profiling runs)")
     ap.add_argument("--heads", type=int, default=0, help="override H (smaller profiling cases)")

@@ -135,6 +135,53 @@ int rehyat_forward_ex(const void* q, const void* k, const void* v,
                       int chunk_frames, int overlap_frames, int sets, int layout,
                       void* out, void* workspace, size_t workspace_bytes, void* stream);
 
+/* Learned feature map ("ReHyAt", §4.3 Training specification and §7.1
+ * Training Details: a two-layer MLP with degree-2 polynomial features,
+ * separate maps for queries and keys; the §3.2 feature-map equation with
+ * P = 2).  Per head h and row x (d wide):
+ *   u   = W2[h] relu(W1[h] x + b1[h]) + b2[h]     (hidden width 2d)
+ *   phi = [1 + elu(u[0:d]), (1 + elu(u[d:2d]))^2]  (2d wide, non-negative)
+ * The pages fix neither the hidden width nor the output non-linearity; this
+ * reading keeps phi non-negative (§3.1) and gives about 2.4 M parameters per
+ * block for 12 heads at d = 128 (the paper's figure).  With W1 = [I; -I],
+ * W2 = [[I, -I]; [I, -I]] and zero biases it is the fixed phi.
+ *   x   [B, H, N, d] or [B, N, H, d] (layout) bf16 device
+ *   W1  [H, 2d, d] bf16, b1 [H, 2d] fp32, W2 [H, 2d, 2d] bf16, b2 [H, 2d] fp32
+ *   phi [B, H, N, 2d] bf16 device, written (caller-owned, 16-byte aligned)
+ * Tensor cores: both GEMMs accumulate in fp32; relu(W1 x + b1) is rounded
+ * to bf16 before the second GEMM and phi to bf16 on output.  d is 64 or
+ * 128.  Returns REHYAT_EINVAL for null / misaligned pointers or bad sizes. */
+int rehyat_phi_mlp(const void* x, int B, int H, int N, int d, int layout,
+                   const void* W1, const float* b1, const void* W2, const float* b2,
+                   void* phi, void* stream);
+
+/* rehyat_forward_ex with precomputed feature maps: phi_q, phi_k are
+ * [B, H, N, 2d] bf16 device (any non-negative map, e.g. rehyat_phi_mlp's
+ * output) used in place of the fixed phi in the linear term and the states:
+ *   a^L = phi_q(q_i) S_t, n^L = phi_q(q_i) z_t, S_t = sum phi_k(k_j) v_j^T,
+ *   z_t = sum phi_k(k_j) over T^L_t.  Workspace as rehyat_forward_ex (same
+ *   size query).  q, k, v, out in `layout`; phi_q / phi_k always [B,H,N,2d]. */
+int rehyat_forward_phi(const void* q, const void* k, const void* v,
+                       const void* phi_q, const void* phi_k,
+                       int B, int H, int F, int S_tok, int d,
+                       int chunk_frames, int overlap_frames, int sets, int layout,
+                       void* out, void* workspace, size_t workspace_bytes, void* stream);
+
+/* The whole hybrid attention with learned feature maps: rehyat_phi_mlp of q
+ * (weights Wq1, bq1, Wq2, bq2) and of k (Wk1, bk1, Wk2, bk2) in one launch
+ * into the workspace, then rehyat_forward_phi.  Weight shapes as
+ * rehyat_phi_mlp.  workspace may be NULL (stream-ordered scratch), else it
+ * holds rehyat_forward_mlp_workspace_bytes(...) bytes, 256-byte aligned. */
+int rehyat_forward_mlp_workspace_bytes(int B, int H, int F, int S_tok, int d,
+                                       int chunk_frames, int overlap_frames, int sets,
+                                       size_t* bytes);
+int rehyat_forward_mlp(const void* q, const void* k, const void* v,
+                       const void* Wq1, const float* bq1, const void* Wq2, const float* bq2,
+                       const void* Wk1, const float* bk1, const void* Wk2, const float* bk2,
+                       int B, int H, int F, int S_tok, int d,
+                       int chunk_frames, int overlap_frames, int sets, int layout,
+                       void* out, void* workspace, size_t workspace_bytes, void* stream);
+
 /* fp32 forward (SIMT fp32 throughout, accurate exp); same sets and layout.
  * Meant for small problems and tight-tolerance checks; any size is legal. */
 int rehyat_forward_f32(const float* q, const float* k, const float* v,

@@ -260,14 +260,18 @@ unsigned long long* g_trace = nullptr;  // cycle-trace buffer of trace builds
 // ---------------------------------------------------------------------------
 // stages
 // ---------------------------------------------------------------------------
+// phi_k (optional): precomputed phi(K) [B, H, N, 2d] of a learned feature map.
 int run_states(const void* k, const void* v, const FwdPlan& P, uint8_t* ws, float* Sf_out, float* z_out,
-               cudaStream_t s) {
+               cudaStream_t s, const void* phi_k = nullptr) {
   float* pS = reinterpret_cast<float*>(ws + P.off_pS);
   float* pz = reinterpret_cast<float*>(ws + P.off_pz);
   if (P.n_seg > 0) {
     StateParams sp;
     std::memset(&sp, 0, sizeof(sp));
-    if (!make_map4(&sp.tm_k, k, P.D, P.N, P.H, P.B, P.rs, P.hs, P.bs, 64) ||
+    const long long D2 = 2LL * P.D;
+    if ((phi_k == nullptr && !make_map4(&sp.tm_k, k, P.D, P.N, P.H, P.B, P.rs, P.hs, P.bs, 64)) ||
+        (phi_k != nullptr &&
+         !make_map4(&sp.tm_phik, phi_k, D2, P.N, P.H, P.B, D2, P.N * D2, P.H * P.N * D2, 64)) ||
         !make_map4(&sp.tm_v, v, P.D, P.N, P.H, P.B, P.rs, P.hs, P.bs, 64))
       return REHYAT_ECUDA;
     sp.sg = SegGeom{P.N, P.chunk_tok, P.ovl_tok, P.n_seg, P.nsplit, 0, 0, P.bidir ? P.S_tok : 0};
@@ -275,7 +279,9 @@ int run_states(const void* k, const void* v, const FwdPlan& P, uint8_t* ws, floa
     sp.H = P.H;
     sp.part_S = pS;
     sp.part_z = pz;
-    int st = cuda_status(launch_chunk_state(P.D, sp, P.BH * P.n_seg * P.nsplit, s));
+    const int n_ctas = P.BH * P.n_seg * P.nsplit;
+    int st = cuda_status(phi_k != nullptr ? launch_chunk_state_phi(P.D, sp, n_ctas, s)
+                                          : launch_chunk_state(P.D, sp, n_ctas, s));
     if (st != REHYAT_OK) return st;
   }
   if (P.bidir) {
@@ -298,8 +304,10 @@ int run_states(const void* k, const void* v, const FwdPlan& P, uint8_t* ws, floa
                                        reinterpret_cast<float*>(ws + P.off_zt), s));
 }
 
+// phi_q (optional): precomputed phi(q) [B, H, N, 2d] of a learned feature map.
 int run_attention(const void* q, const void* k, const void* v, const FwdPlan& P, uint8_t* ws, void* out,
-                  float* aS, float* nS, float* aL, float* nL, float* Mo, cudaStream_t s) {
+                  float* aS, float* nS, float* aL, float* nL, float* Mo, cudaStream_t s,
+                  const void* phi_q = nullptr) {
   AttnParams ap;
   std::memset(&ap, 0, sizeof(ap));
   if (!make_map4(&ap.tm_q, q, P.D, P.N, P.H, P.B, P.rs, P.hs, P.bs, 128) ||
@@ -325,7 +333,57 @@ int run_attention(const void* q, const void* k, const void* v, const FwdPlan& P,
 #ifdef REHYAT_TRACE
   ap.trace = g_trace;
 #endif
+  if (phi_q != nullptr) {
+    ap.phi_q = static_cast<const __nv_bfloat16*>(phi_q);
+    return cuda_status(launch_attention_phi(P.D, ap, P.n_units, s));
+  }
   return cuda_status(launch_attention(P.D, aS != nullptr, ap, P.n_units, s));
+}
+
+// Learned feature maps of up to two inputs (q then k) in one launch; every
+// x is [B, N, H, d] or [B, H, N, d] by (rs, hs, bs), every phi [B, H, N, 2d].
+struct MlpArgs {
+  const void* x;
+  const void* W1;
+  const float* b1;
+  const void* W2;
+  const float* b2;
+  void* phi;
+};
+
+int check_mlp_args(const MlpArgs& a) {
+  if (check_ptr(a.x) || check_ptr(a.W1) || check_ptr(a.b1) || check_ptr(a.W2) || check_ptr(a.b2) ||
+      check_ptr(a.phi))
+    return REHYAT_EINVAL;
+  return REHYAT_OK;
+}
+
+int run_phi_mlp(const MlpArgs* maps, int n_maps, int B, int H, int N, int d, long long rs, long long hs,
+                long long bs, cudaStream_t s) {
+  MlpParams mp;
+  std::memset(&mp, 0, sizeof(mp));
+  const long long D2 = 2LL * d;
+  for (int i = 0; i < n_maps; ++i) {
+    if (!make_map4(&mp.tm_x[i], maps[i].x, d, N, H, B, rs, hs, bs, 128) ||
+        !make_map(&mp.tm_w1[i], maps[i].W1, d, D2, H, static_cast<int>(D2)) ||
+        !make_map(&mp.tm_w2[i], maps[i].W2, D2, D2, H, static_cast<int>(D2)))
+      return REHYAT_ECUDA;
+    mp.b1[i] = maps[i].b1;
+    mp.b2[i] = maps[i].b2;
+    mp.phi[i] = static_cast<__nv_bfloat16*>(maps[i].phi);
+  }
+  mp.N = N;
+  mp.H = H;
+  mp.BH = B * H;
+  // one wave of CTAs over the (map, bh) pairs, each walking its share of the
+  // 128-row tiles with the head's weights loaded once
+  const int pairs = n_maps * mp.BH;
+  const int ntiles = cdiv(N, 128);
+  int groups = kSplitTarget / pairs;
+  groups = groups < 1 ? 1 : (groups > ntiles ? ntiles : groups);
+  if (static_cast<long long>(pairs) * groups > INT_MAX) return REHYAT_EINVAL;
+  mp.groups = groups;
+  return cuda_status(launch_phi_mlp(d, mp, n_maps, s));
 }
 
 struct WsGuard {  // stream-ordered scratch owned by one call
@@ -461,6 +519,104 @@ REHYAT_API int rehyat_forward_ex(const void* q, const void* k, const void* v, in
   st = run_states(k, v, P, w, nullptr, nullptr, s);
   if (st != REHYAT_OK) return st;
   return run_attention(q, k, v, P, w, out, nullptr, nullptr, nullptr, nullptr, nullptr, s);
+}
+
+REHYAT_API int rehyat_phi_mlp(const void* x, int B, int H, int N, int d, int layout, const void* W1,
+                              const float* b1, const void* W2, const float* b2, void* phi, void* stream) {
+  if (B < 1 || H < 1 || N < 1) return REHYAT_EINVAL;
+  int st = check_d(d);
+  if (st != REHYAT_OK) return st;
+  if (static_cast<long long>(B) * H > INT_MAX / 2 || static_cast<long long>(B) * H * N * d > (1LL << 46))
+    return REHYAT_EINVAL;
+  const long long Nl = N, dl = d, Hl = H;
+  long long rs, hs, bs;
+  if (layout == REHYAT_LAYOUT_BHND) {
+    rs = dl; hs = Nl * dl; bs = Hl * Nl * dl;
+  } else if (layout == REHYAT_LAYOUT_BNHD) {
+    rs = Hl * dl; hs = dl; bs = Nl * Hl * dl;
+  } else {
+    return REHYAT_EINVAL;
+  }
+  const MlpArgs a{x, W1, b1, W2, b2, phi};
+  if (check_mlp_args(a)) return REHYAT_EINVAL;
+  return run_phi_mlp(&a, 1, B, H, N, d, rs, hs, bs, static_cast<cudaStream_t>(stream));
+}
+
+REHYAT_API int rehyat_forward_phi(const void* q, const void* k, const void* v, const void* phi_q, const void* phi_k,
+                                  int B, int H, int F, int S_tok, int d, int chunk_frames, int overlap_frames,
+                                  int sets, int layout, void* out, void* workspace, size_t workspace_bytes,
+                                  void* stream) {
+  FwdPlan P;
+  int st = plan_forward_sets(B, H, F, S_tok, d, chunk_frames, overlap_frames, sets, &P);
+  if (st != REHYAT_OK) return st;
+  st = apply_layout(layout, &P);
+  if (st != REHYAT_OK) return st;
+  if (check_qkvo(q, k, v, out) || check_ptr(phi_q) || check_ptr(phi_k)) return REHYAT_EINVAL;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  WsGuard own(s);
+  if (workspace == nullptr) {
+    st = own.alloc(P.bytes);
+    if (st != REHYAT_OK) return st;
+    workspace = own.p;
+  } else {
+    if (reinterpret_cast<uintptr_t>(workspace) % 256 != 0) return REHYAT_EINVAL;
+    if (workspace_bytes < P.bytes) return REHYAT_ENOMEM;
+  }
+  uint8_t* w = static_cast<uint8_t*>(workspace);
+  st = run_states(k, v, P, w, nullptr, nullptr, s, phi_k);
+  if (st != REHYAT_OK) return st;
+  return run_attention(q, k, v, P, w, out, nullptr, nullptr, nullptr, nullptr, nullptr, s, phi_q);
+}
+
+namespace {
+// Workspace of the learned-map forward: phi(q), phi(k), then the forward's.
+size_t mlp_phi_bytes(const FwdPlan& P) { return align256(static_cast<size_t>(P.BH) * P.N * 2 * P.D * 2); }
+}  // namespace
+
+REHYAT_API int rehyat_forward_mlp_workspace_bytes(int B, int H, int F, int S_tok, int d, int chunk_frames,
+                                                  int overlap_frames, int sets, size_t* bytes) {
+  if (bytes == nullptr) return REHYAT_EINVAL;
+  FwdPlan P;
+  int st = plan_forward_sets(B, H, F, S_tok, d, chunk_frames, overlap_frames, sets, &P);
+  if (st != REHYAT_OK) return st;
+  *bytes = 2 * mlp_phi_bytes(P) + P.bytes;
+  return REHYAT_OK;
+}
+
+REHYAT_API int rehyat_forward_mlp(const void* q, const void* k, const void* v, const void* Wq1, const float* bq1,
+                                  const void* Wq2, const float* bq2, const void* Wk1, const float* bk1,
+                                  const void* Wk2, const float* bk2, int B, int H, int F, int S_tok, int d,
+                                  int chunk_frames, int overlap_frames, int sets, int layout, void* out,
+                                  void* workspace, size_t workspace_bytes, void* stream) {
+  FwdPlan P;
+  int st = plan_forward_sets(B, H, F, S_tok, d, chunk_frames, overlap_frames, sets, &P);
+  if (st != REHYAT_OK) return st;
+  st = apply_layout(layout, &P);
+  if (st != REHYAT_OK) return st;
+  if (check_qkvo(q, k, v, out)) return REHYAT_EINVAL;
+  const void* wts[8] = {Wq1, bq1, Wq2, bq2, Wk1, bk1, Wk2, bk2};
+  for (const void* w : wts)
+    if (check_ptr(w)) return REHYAT_EINVAL;
+  const size_t phi_bytes = mlp_phi_bytes(P);
+  const size_t need = 2 * phi_bytes + P.bytes;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  WsGuard own(s);
+  if (workspace == nullptr) {
+    st = own.alloc(need);
+    if (st != REHYAT_OK) return st;
+    workspace = own.p;
+  } else {
+    if (reinterpret_cast<uintptr_t>(workspace) % 256 != 0) return REHYAT_EINVAL;
+    if (workspace_bytes < need) return REHYAT_ENOMEM;
+  }
+  uint8_t* w = static_cast<uint8_t*>(workspace);
+  const MlpArgs maps[2] = {{q, Wq1, bq1, Wq2, bq2, w}, {k, Wk1, bk1, Wk2, bk2, w + phi_bytes}};
+  st = run_phi_mlp(maps, 2, P.B, P.H, P.N, P.D, P.rs, P.hs, P.bs, s);
+  if (st != REHYAT_OK) return st;
+  uint8_t* fw = w + 2 * phi_bytes;
+  st = run_states(k, v, P, fw, nullptr, nullptr, s, w + phi_bytes);
+  if (st != REHYAT_OK) return st;
+  return run_attention(q, k, v, P, fw, out, nullptr, nullptr, nullptr, nullptr, nullptr, s, w);
 }
 
 REHYAT_API int rehyat_forward_parts(const void* q, const void* k, const void* v, int B, int H, int F, int S_tok,

@@ -6,7 +6,10 @@
 //    sets: exact softmax over the chunk's window [lo_t, hi_t) plus the linear
 //    term phi(q) S_t, phi(q) z_t of every earlier key (§3.1 caching).
 // 2. phi_state_kernel: phi(K)^T V and sum phi(K) per key segment (the two
-//    query-independent sums of §3.1), phi of §3.2 with P = 2, psi = 1 + elu.
+//    query-independent sums of §3.1), phi of §3.2 with P = 2, psi = 1 + elu,
+//    or precomputed phi(K) of a learned map.
+// 3. phi_mlp_kernel: the learned feature map (two-layer MLP, degree-2
+//    polynomial features; §4.3 Training specification, §7.1).
 //
 // Layout conventions (all operand tiles use the 128-byte TMA swizzle):
 //   a "box" is 128 B wide (64 bf16) and R rows tall; row r lives at r*128 and
@@ -162,7 +165,9 @@ constexpr int TRACE_CTAS = 4, TRACE_EVENTS = 16, TRACE_TILES = 64;
 // 10+X P_X seen, 12+X S_X(j+1) issued, 14 unit start (j = 0), Q and K_0 in
 // (j = 1), K_{j+1} in (j + 2), 15 P_A.V_j issued
 
-template <int D, bool PARTS>
+// PHI: the linear term takes phi(q) rows precomputed by a learned feature map
+// (p.phi_q) instead of evaluating the fixed phi on the Q tile.
+template <int D, bool PARTS, bool PHI>
 __global__ void __launch_bounds__(384, 1) hybrid_chunk_attn_kernel(const __grid_constant__ AttnParams p) {
   using C = AttnCfg<D>;
   constexpr int NS = C::NSLOTS;
@@ -367,6 +372,36 @@ __global__ void __launch_bounds__(384, 1) hybrid_chunk_attn_kernel(const __grid_
       if (has_lin && ok) {
         const float sc = ex2(-m_used);  // exp(-M), <= 1
         const float* zp = p.z + bh * p.z_bh + t * p.z_t;
+        if constexpr (PHI) {
+          // phi(q) row of 2D bf16 features: [0, D) into columns [0, D/2),
+          // [D, 2D) into [D/2, D), two features a column
+          const uint4* fr = reinterpret_cast<const uint4*>(p.phi_q) +
+                            (static_cast<size_t>(bh) * p.g.N_q + (vrow ? qrow : 0)) * (2 * D / 8);
+#pragma unroll
+          for (int b = 0; b < C::NBOX; ++b) {
+            uint32_t pa[32], pb[32];
+#pragma unroll
+            for (int cc = 0; cc < 8; ++cc) {
+              const uint4 z4 = make_uint4(0u, 0u, 0u, 0u);
+              const uint4 ra = vrow ? __ldg(fr + 8 * b + cc) : z4;
+              const uint4 rb = vrow ? __ldg(fr + D / 8 + 8 * b + cc) : z4;
+              const uint32_t wa[4] = {ra.x, ra.y, ra.z, ra.w};
+              const uint32_t wb[4] = {rb.x, rb.y, rb.z, rb.w};
+#pragma unroll
+              for (int h = 0; h < 4; ++h) {
+                const int dim = 64 * b + 8 * cc + 2 * h;
+                const uint32_t ua = pack_bf16(bf16lo(wa[h]) * sc, bf16hi(wa[h]) * sc);
+                const uint32_t ub = pack_bf16(bf16lo(wb[h]) * sc, bf16hi(wb[h]) * sc);
+                nl += bf16lo(ua) * zp[dim] + bf16hi(ua) * zp[dim + 1] + bf16lo(ub) * zp[D + dim] +
+                      bf16hi(ub) * zp[D + dim + 1];
+                pa[cc * 4 + h] = ua;
+                pb[cc * 4 + h] = ub;
+              }
+            }
+            tmem_st32(tS + 32 * b, pa);
+            tmem_st32(tS + D / 2 + 32 * b, pb);
+          }
+        } else {
         const uint8_t* qrow = smem + C::OFF_Q + X * C::TILE_BYTES + r * 128;
 #pragma unroll
         for (int b = 0; b < C::NBOX; ++b) {
@@ -393,6 +428,7 @@ __global__ void __launch_bounds__(384, 1) hybrid_chunk_attn_kernel(const __grid_
           // features psi (0..D-1) then psi^2 (D..2D-1), two per column
           tmem_st32(tS + 32 * b, pa);
           tmem_st32(tS + D / 2 + 32 * b, pb);
+        }
         }
         warp_release(BAR(C::B_PHI + X), lane);
         ok = warp_wait(BAR(C::B_LIN + X), 0, abort);
@@ -644,7 +680,10 @@ struct StCfg {
   static_assert(G * 2 * D * 4 <= STAGE, "z reduction scratch");
 };
 
-template <int D>
+// PRE: phi(K) is precomputed (a learned feature map) and arrives by TMA
+// through p.tm_phik straight into the A-operand layout; the phi warps then
+// only zero the rows past the piece's end and sum phi(K).
+template <int D, bool PRE>
 __global__ void __launch_bounds__(StCfg<D>::THREADS, 1) phi_state_kernel(const __grid_constant__ StateParams p) {
   using C = StCfg<D>;
   extern __shared__ uint8_t smem_raw[];
@@ -684,7 +723,10 @@ __global__ void __launch_bounds__(StCfg<D>::THREADS, 1) phi_state_kernel(const _
     fence_mbar_init();
   }
   if (warp == C::PHI_WARPS && lane == 0) {
-    prefetch_tmap(&p.tm_k);
+    if (PRE)
+      prefetch_tmap(&p.tm_phik);
+    else
+      prefetch_tmap(&p.tm_k);
     prefetch_tmap(&p.tm_v);
   }
   if (warp == C::PHI_WARPS + 1) {
@@ -720,6 +762,27 @@ __global__ void __launch_bounds__(StCfg<D>::THREADS, 1) phi_state_kernel(const _
         const bool valid = a + 64 * i + tok < b;
         const int off = tok * 128 + ((cc ^ (tok & 7)) << 4);
         uint4 pa = make_uint4(0u, 0u, 0u, 0u), pb = pa;
+        if (PRE) {
+          uint4* fa = reinterpret_cast<uint4*>(ph + bx * C::BOX + off);
+          uint4* fb = reinterpret_cast<uint4*>(ph + (C::NBOX + bx) * C::BOX + off);
+          if (valid) {
+            pa = *fa;
+            pb = *fb;
+            const uint32_t va[4] = {pa.x, pa.y, pa.z, pa.w};
+            const uint32_t vb[4] = {pb.x, pb.y, pb.z, pb.w};
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+              za[2 * h] = add_bf16_lo(va[h], za[2 * h]);
+              za[2 * h + 1] = add_bf16_hi(va[h], za[2 * h + 1]);
+              zb[2 * h] = add_bf16_lo(vb[h], zb[2 * h]);
+              zb[2 * h + 1] = add_bf16_hi(vb[h], zb[2 * h + 1]);
+            }
+          } else {  // a later segment's token: out of this piece's sums
+            *fa = pa;
+            *fb = pb;
+          }
+          continue;
+        }
         if (valid) {
           const uint4 raw = *reinterpret_cast<const uint4*>(kt + bx * C::BOX + off);
           const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
@@ -798,12 +861,17 @@ __global__ void __launch_bounds__(StCfg<D>::THREADS, 1) phi_state_kernel(const _
         ok = mbar_wait(BAR(C::B_EMPTY + st), ((i / C::NST) & 1) ^ 1, abort);
         if (!ok) break;
         const uint32_t base = smem_u32(smem + st * C::STAGE);
-        mbar_arrive_expect_tx(BAR(C::B_KV + st), 2 * C::KV_BYTES);
+        mbar_arrive_expect_tx(BAR(C::B_KV + st), PRE ? C::KV_BYTES + C::PHI_BYTES : 2 * C::KV_BYTES);
         for (int bb = 0; bb < C::NBOX; ++bb) {
-          tma_load_4d(base + bb * C::BOX, &p.tm_k, BAR(C::B_KV + st), 64 * bb, a + 64 * i, bh % p.H, bh / p.H);
+          if (!PRE)
+            tma_load_4d(base + bb * C::BOX, &p.tm_k, BAR(C::B_KV + st), 64 * bb, a + 64 * i, bh % p.H, bh / p.H);
           tma_load_4d(base + C::KV_BYTES + bb * C::BOX, &p.tm_v, BAR(C::B_KV + st), 64 * bb, a + 64 * i, bh % p.H,
                       bh / p.H);
         }
+        if (PRE)
+          for (int bb = 0; bb < 2 * C::NBOX; ++bb)
+            tma_load_4d(base + 2 * C::KV_BYTES + bb * C::BOX, &p.tm_phik, BAR(C::B_KV + st), 64 * bb, a + 64 * i,
+                        bh % p.H, bh / p.H);
       }
       for (int i2 = (i > C::NST ? i - C::NST : 0); i2 < i; ++i2)
         drain_wait(BAR(C::B_KV + i2 % C::NST), (i2 / C::NST) & 1);
@@ -838,6 +906,241 @@ __global__ void __launch_bounds__(StCfg<D>::THREADS, 1) phi_state_kernel(const _
   tc_fence_before();
   __syncthreads();
   if (warp == C::PHI_WARPS + 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+// ============================================================================
+// Learned feature map: phi = [psi(u_1), psi(u_2)^2], u = W2 relu(W1 x + b1) + b2
+// ============================================================================
+// Two chained GEMMs per 128-row tile, both on the tensor cores with the
+// head's weights resident in shared memory for the CTA's whole life:
+//   H = x W1^T          (SS MMA, M = 128, N = 2D, K = D)    -> TMEM [0, 2D)
+//   R = relu(H + b1)    bf16, written back into TMEM over H's columns
+//   U = R W2^T          (TS MMA, M = 128, N = 2D, K = 2D)   -> TMEM [2D, 4D)
+//   phi = [1 + elu(U_1 + b2_1), (1 + elu(U_2 + b2_2))^2]   bf16 -> global
+// Warps 0-7 run both epilogues (warps w and w + 4 share TMEM lanes and split
+// the columns: group 0 the first half of H and U, group 1 the second); warp 8
+// is the TMA producer, warp 9 the MMA issuer.  The x tile is released as soon
+// as its GEMM has read it, so the next tile's load overlaps both epilogues,
+// and the next H GEMM runs while the epilogue still reads U.
+template <int D>
+struct MlpCfg {
+  static constexpr int HID = 2 * D;                 // hidden width
+  static constexpr int OUT = 2 * D;                 // feature width D'
+  static constexpr int NBX = D / 64;                // 64-column boxes across x and W1
+  static constexpr int NBH = HID / 64;              // ... across the hidden units (W2)
+  static constexpr int XBOX = 128 * 128;            // 128 rows x 128 B
+  static constexpr int X_BYTES = NBX * XBOX;
+  static constexpr int W1BOX = HID * 128;           // HID rows x 128 B
+  static constexpr int W2BOX = OUT * 128;
+  static constexpr int W1_BYTES = NBX * W1BOX;
+  static constexpr int W2_BYTES = NBH * W2BOX;
+  static constexpr int NXB = (D == 128) ? 1 : 2;    // x tile buffers (the weights fill the rest)
+  static constexpr int OFF_W1 = 0;
+  static constexpr int OFF_W2 = W1_BYTES;
+  static constexpr int OFF_X = OFF_W2 + W2_BYTES;
+  static constexpr int OFF_BAR = OFF_X + NXB * X_BYTES;
+  static constexpr int SMEM = OFF_BAR + 256 + 1024;
+  static constexpr uint32_t TMEM_COLS = (HID + OUT <= 256) ? 256u : 512u;
+  static constexpr int EPI_WARPS = 8;
+  static constexpr int THREADS = 32 * EPI_WARPS + 64;
+  static constexpr int B_W = 0, B_X = 1, B_XE = 1 + NXB, B_H = 1 + 2 * NXB, B_R = B_H + 1, B_U = B_H + 2,
+                       B_UE = B_H + 3, B_FIN = B_H + 4;
+  // both GEMMs: A and B K-major (x rows / R rows by W rows)
+  static constexpr uint32_t IDESC1 = idesc_bf16_f32(128, HID, 0, 0);
+  static constexpr uint32_t IDESC2 = idesc_bf16_f32(128, OUT, 0, 0);
+  static_assert(SMEM <= 232448, "shared memory");
+  static_assert((B_FIN + 1) * 8 <= 128, "barrier area");
+  static_assert(HID + OUT <= 512, "tensor memory");
+};
+
+template <int D>
+__global__ void __launch_bounds__(MlpCfg<D>::THREADS, 1) phi_mlp_kernel(const __grid_constant__ MlpParams p) {
+  using C = MlpCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int grp_id = blockIdx.x % p.groups;  // CTA = (map, bh, row group)
+  const int rest = blockIdx.x / p.groups;
+  const int bh = rest % p.BH;
+  const int m = rest / p.BH;
+  const int hh = bh % p.H, bb = bh / p.H;
+  const int ntiles = cdiv(p.N, 128);
+  const int my_tiles = grp_id < ntiles ? cdiv(ntiles - grp_id, p.groups) : 0;
+  if (my_tiles == 0) return;  // uniform exit, before any barrier or TMEM use
+
+  uint8_t* barea = smem + C::OFF_BAR;
+  const uint32_t bar0 = smem_u32(barea);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(barea + 128);
+  volatile int* abort = reinterpret_cast<volatile int*>(barea + 132);
+#define BAR(i) (bar0 + 8u * static_cast<uint32_t>(i))
+  if (threadIdx.x == 0) {
+    mbar_init(BAR(C::B_W), 1);
+    for (int i = 0; i < C::NXB; ++i) {
+      mbar_init(BAR(C::B_X + i), 1);
+      mbar_init(BAR(C::B_XE + i), 1);
+    }
+    mbar_init(BAR(C::B_H), 1);
+    mbar_init(BAR(C::B_R), C::EPI_WARPS);
+    mbar_init(BAR(C::B_U), 1);
+    mbar_init(BAR(C::B_UE), C::EPI_WARPS);
+    mbar_init(BAR(C::B_FIN), 1);
+    *abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == C::EPI_WARPS && lane == 0) {
+    prefetch_tmap(&p.tm_x[m]);
+    prefetch_tmap(&p.tm_w1[m]);
+    prefetch_tmap(&p.tm_w2[m]);
+  }
+  if (warp == C::EPI_WARPS + 1) {
+    tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp < C::EPI_WARPS) {
+    // ============================ epilogues ============================
+    const int quarter = warp & 3, g = warp >> 2;
+    const uint32_t lane_off = static_cast<uint32_t>(32 * quarter) << 16;
+    const float4* b1 = reinterpret_cast<const float4*>(p.b1[m] + hh * C::HID + g * D);  // group's hidden units
+    const float4* b2 = reinterpret_cast<const float4*>(p.b2[m] + hh * C::OUT + g * D);  // group's features
+    bool ok = true;
+    for (int it = 0; it < my_tiles; ++it) {
+      const int tile = grp_id + it * p.groups;
+      ok = warp_wait(BAR(C::B_H), it & 1, abort);
+      if (!ok) break;
+      tc_fence_after();
+      // R = relu(H + b1) as bf16 pairs: the group's D hidden units go to the
+      // first D/2 of its own D columns (chunk c is read before any column it
+      // overwrites, and the two groups' column ranges are disjoint)
+#pragma unroll 1
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t v[32];
+        tmem_ld32(tmem + lane_off + g * D + 32 * c, v);
+        tmem_ld_wait();
+        reg_fence(v);
+        uint32_t r[16];
+#pragma unroll
+        for (int q4 = 0; q4 < 8; ++q4) {
+          const float4 bv = __ldg(b1 + 8 * c + q4);
+          r[2 * q4] = pack_bf16(fmaxf(__uint_as_float(v[4 * q4]) + bv.x, 0.f),
+                                fmaxf(__uint_as_float(v[4 * q4 + 1]) + bv.y, 0.f));
+          r[2 * q4 + 1] = pack_bf16(fmaxf(__uint_as_float(v[4 * q4 + 2]) + bv.z, 0.f),
+                                    fmaxf(__uint_as_float(v[4 * q4 + 3]) + bv.w, 0.f));
+        }
+        tmem_st16(tmem + lane_off + g * D + 16 * c, r);
+      }
+      warp_release(BAR(C::B_R), lane);
+      ok = warp_wait(BAR(C::B_U), it & 1, abort);
+      if (!ok) break;
+      tc_fence_after();
+      // phi = psi(U + b2) (group 0) or its square (group 1), one row a thread
+      const int row = tile * 128 + 32 * quarter + lane;
+      const bool vrow = row < p.N;
+      uint4* dst = reinterpret_cast<uint4*>(p.phi[m] + (static_cast<size_t>(bh) * p.N + (vrow ? row : 0)) * C::OUT +
+                                            g * D);
+#pragma unroll 1
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t v[32];
+        tmem_ld32(tmem + lane_off + C::HID + g * D + 32 * c, v);
+        tmem_ld_wait();
+        reg_fence(v);
+        uint32_t o[16];
+#pragma unroll
+        for (int q4 = 0; q4 < 8; ++q4) {
+          const float4 bv = __ldg(b2 + 8 * c + q4);
+          float f0 = psi1(__uint_as_float(v[4 * q4]) + bv.x);
+          float f1 = psi1(__uint_as_float(v[4 * q4 + 1]) + bv.y);
+          float f2 = psi1(__uint_as_float(v[4 * q4 + 2]) + bv.z);
+          float f3 = psi1(__uint_as_float(v[4 * q4 + 3]) + bv.w);
+          if (g) {
+            f0 *= f0;
+            f1 *= f1;
+            f2 *= f2;
+            f3 *= f3;
+          }
+          o[2 * q4] = pack_bf16(f0, f1);
+          o[2 * q4 + 1] = pack_bf16(f2, f3);
+        }
+        if (vrow)
+#pragma unroll
+          for (int k4 = 0; k4 < 4; ++k4) dst[4 * c + k4] = make_uint4(o[4 * k4], o[4 * k4 + 1], o[4 * k4 + 2], o[4 * k4 + 3]);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(BAR(C::B_UE));
+    }
+  } else if (warp == C::EPI_WARPS) {
+    // =========================== TMA producer ===========================
+    if (lane == 0) {
+      mbar_arrive_expect_tx(BAR(C::B_W), C::W1_BYTES + C::W2_BYTES);
+      for (int b = 0; b < C::NBX; ++b)
+        tma_load_3d(smem_u32(smem + C::OFF_W1 + b * C::W1BOX), &p.tm_w1[m], BAR(C::B_W), 64 * b, 0, hh);
+      for (int b = 0; b < C::NBH; ++b)
+        tma_load_3d(smem_u32(smem + C::OFF_W2 + b * C::W2BOX), &p.tm_w2[m], BAR(C::B_W), 64 * b, 0, hh);
+      bool ok = true;
+      int it = 0;
+      for (; it < my_tiles && ok; ++it) {
+        const int slot = it % C::NXB;
+        ok = mbar_wait(BAR(C::B_XE + slot), ((it / C::NXB) & 1) ^ 1, abort);
+        if (!ok) break;
+        const uint32_t dst = smem_u32(smem + C::OFF_X + slot * C::X_BYTES);
+        mbar_arrive_expect_tx(BAR(C::B_X + slot), C::X_BYTES);
+        for (int b = 0; b < C::NBX; ++b)
+          tma_load_4d(dst + b * C::XBOX, &p.tm_x[m], BAR(C::B_X + slot), 64 * b, 128 * (grp_id + it * p.groups), hh,
+                      bb);
+      }
+      drain_wait(BAR(C::B_W), 0);
+      for (int i2 = (it > C::NXB ? it - C::NXB : 0); i2 < it; ++i2)
+        drain_wait(BAR(C::B_X + i2 % C::NXB), (i2 / C::NXB) & 1);
+    }
+  } else {
+    // ============================ MMA issuer ============================
+    if (lane == 0) {
+      constexpr uint32_t HI = desc_hi_sw128(1024);  // K-major: 8-row groups 1024 B apart
+      const uint32_t lo_w1 = desc_lo(smem_u32(smem + C::OFF_W1), 16);
+      const uint32_t lo_w2 = desc_lo(smem_u32(smem + C::OFF_W2), 16);
+      bool ok = mbar_wait(BAR(C::B_W), 0, abort);
+      for (int it = 0; it < my_tiles && ok; ++it) {
+        const int slot = it % C::NXB;
+        ok = mbar_wait(BAR(C::B_X + slot), (it / C::NXB) & 1, abort);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t lo_x = desc_lo(smem_u32(smem + C::OFF_X + slot * C::X_BYTES), 16);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk)  // K-step kk: box kk/4, 32 B into the swizzled row
+          mma_ss(tmem, desc_join(lo_x + (((kk >> 2) * C::XBOX + (kk & 3) * 32) >> 4), HI),
+                 desc_join(lo_w1 + (((kk >> 2) * C::W1BOX + (kk & 3) * 32) >> 4), HI), C::IDESC1, kk > 0 ? 1u : 0u);
+        mma_commit(BAR(C::B_XE + slot));
+        mma_commit(BAR(C::B_H));
+        // R of this tile written, and U free (the previous tile's features stored)
+        ok = mbar_wait(BAR(C::B_R), it & 1, abort) && mbar_wait(BAR(C::B_UE), (it & 1) ^ 1, abort);
+        if (!ok) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < C::HID / 16; ++kk) {  // 16 hidden units = 8 packed columns of R
+          const uint32_t a = tmem + (kk / (D / 16)) * D + (kk % (D / 16)) * 8;
+          mma_ts(tmem + C::HID, a, desc_join(lo_w2 + (((kk >> 2) * C::W2BOX + (kk & 3) * 32) >> 4), HI), C::IDESC2,
+                 kk > 0 ? 1u : 0u);
+        }
+        mma_commit(BAR(C::B_U));
+      }
+      mma_commit(BAR(C::B_FIN));
+      drain_wait(BAR(C::B_FIN), 0);
+    }
+  }
+#undef BAR
+  tc_fence_before();
+  __syncthreads();
+  if (warp == C::EPI_WARPS + 1) {
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
   }
@@ -974,9 +1277,9 @@ int grid_for(long long n, int threads) {
 int attn_smem_bytes(int D) { return D == 128 ? AttnCfg<128>::SMEM : AttnCfg<64>::SMEM; }
 int state_smem_bytes(int D) { return D == 128 ? StCfg<128>::SMEM : StCfg<64>::SMEM; }
 
-template <int D, bool PARTS>
+template <int D, bool PARTS, bool PHI = false>
 static cudaError_t launch_attn_t(const AttnParams& p, int n_units, cudaStream_t s) {
-  auto* k = hybrid_chunk_attn_kernel<D, PARTS>;
+  auto* k = hybrid_chunk_attn_kernel<D, PARTS, PHI>;
   // The in-kernel register split assumes exactly REGS_LAUNCH registers per
   // thread at launch; with fewer, a warpgroup's increase could never be met.
   cudaFuncAttributes fa;
@@ -995,9 +1298,14 @@ cudaError_t launch_attention(int D, bool parts, const AttnParams& p, int n_units
   return parts ? launch_attn_t<64, true>(p, n_units, s) : launch_attn_t<64, false>(p, n_units, s);
 }
 
-template <int D>
+cudaError_t launch_attention_phi(int D, const AttnParams& p, int n_units, cudaStream_t s) {
+  if (n_units <= 0) return cudaSuccess;
+  return D == 128 ? launch_attn_t<128, false, true>(p, n_units, s) : launch_attn_t<64, false, true>(p, n_units, s);
+}
+
+template <int D, bool PRE = false>
 static cudaError_t launch_state_t(const StateParams& p, int n_ctas, cudaStream_t s) {
-  auto* k = phi_state_kernel<D>;
+  auto* k = phi_state_kernel<D, PRE>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, StCfg<D>::SMEM);
   if (e != cudaSuccess) return e;
   k<<<n_ctas, StCfg<D>::THREADS, StCfg<D>::SMEM, s>>>(p);
@@ -1007,6 +1315,11 @@ static cudaError_t launch_state_t(const StateParams& p, int n_ctas, cudaStream_t
 cudaError_t launch_chunk_state(int D, const StateParams& p, int n_ctas, cudaStream_t s) {
   if (n_ctas <= 0) return cudaSuccess;
   return D == 128 ? launch_state_t<128>(p, n_ctas, s) : launch_state_t<64>(p, n_ctas, s);
+}
+
+cudaError_t launch_chunk_state_phi(int D, const StateParams& p, int n_ctas, cudaStream_t s) {
+  if (n_ctas <= 0) return cudaSuccess;
+  return D == 128 ? launch_state_t<128, true>(p, n_ctas, s) : launch_state_t<64, true>(p, n_ctas, s);
 }
 
 cudaError_t launch_state_scan(const float* part_S, const float* part_z, int BH, int n_seg, int nsplit,
@@ -1032,6 +1345,20 @@ cudaError_t launch_state_accumulate(const float* part_S, const float* part_z, in
   const long long n = static_cast<long long>(BH) * 2 * D * (D + 1);
   state_accumulate_kernel<<<grid_for(n, 256), 256, 0, s>>>(part_S, part_z, BH, nsplit, D, state_S, state_z);
   return cudaGetLastError();
+}
+
+template <int D>
+static cudaError_t launch_mlp_t(const MlpParams& p, int n_maps, cudaStream_t s) {
+  auto* k = phi_mlp_kernel<D>;
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, MlpCfg<D>::SMEM);
+  if (e != cudaSuccess) return e;
+  k<<<n_maps * p.BH * p.groups, MlpCfg<D>::THREADS, MlpCfg<D>::SMEM, s>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_phi_mlp(int D, const MlpParams& p, int n_maps, cudaStream_t s) {
+  if (p.N <= 0 || n_maps <= 0) return cudaSuccess;
+  return D == 128 ? launch_mlp_t<128>(p, n_maps, s) : launch_mlp_t<64>(p, n_maps, s);
 }
 
 cudaError_t launch_exp2_fma(const float* x, float* y, long long n, cudaStream_t s) {

@@ -14,6 +14,16 @@ be regenerated alone for sampled-row checks):
           softmax branch dominate, or the linear one, in targeted tests)
   storage: float32, then bfloat16 by round-to-nearest-even (torch's cast).
 Heads are generated in parallel threads; the result does not depend on that.
+
+Learned feature-map weights (make_mlp_weights; the trained weights of the
+paper are not available, so they are drawn): per map (q or k) and head,
+  stream = default_rng(SeedSequence([seed, 10 + which, h]))
+  "near_identity": W1 = [I; -I] + noise/sqrt(d), W2 = [[I, -I]; [I, -I]]
+                   + noise/sqrt(2d) (the weights with which the map is the
+                   fixed 1 + elu features, the natural start of a
+                   distillation), biases noise * 0.1 * N(0, 1)
+  "random":        W1 = N(0,1)/sqrt(d), W2 = N(0,1)/sqrt(2d), biases 0.1 N(0,1)
+  W1, W2 stored bf16, b1, b2 fp32.
 """
 from __future__ import annotations
 
@@ -74,3 +84,29 @@ def make_state(B: int, H: int, d: int, seed: int, scale: float = 1.0):
     S = rng.standard_normal((B, H, 2 * d, d)) * scale
     z = np.abs(rng.standard_normal((B, H, 2 * d))) * scale + 1.0
     return torch.from_numpy(S.astype(np.float32)), torch.from_numpy(z.astype(np.float32))
+
+
+def make_mlp_weights(H: int, d: int, seed: int, which: str = "q", kind: str = "near_identity",
+                     noise: float = 0.1):
+    """Host (W1 [H,2d,d] bf16, b1 [H,2d] fp32, W2 [H,2d,2d] bf16, b2 [H,2d] fp32)."""
+    W1 = np.empty((H, 2 * d, d))
+    W2 = np.empty((H, 2 * d, 2 * d))
+    b1 = np.empty((H, 2 * d))
+    b2 = np.empty((H, 2 * d))
+    I = np.eye(d)
+    for h in range(H):
+        rng = np.random.default_rng(np.random.SeedSequence([seed, 10 + WHICH[which], h]))
+        n1 = rng.standard_normal((2 * d, d)) / np.sqrt(d)
+        n2 = rng.standard_normal((2 * d, 2 * d)) / np.sqrt(2 * d)
+        c1 = rng.standard_normal(2 * d) * 0.1
+        c2 = rng.standard_normal(2 * d) * 0.1
+        if kind == "near_identity":
+            W1[h] = np.concatenate([I, -I], axis=0) + noise * n1
+            W2[h] = np.concatenate([np.concatenate([I, -I], axis=1)] * 2, axis=0) + noise * n2
+            b1[h], b2[h] = noise * c1, noise * c2
+        elif kind == "random":
+            W1[h], W2[h], b1[h], b2[h] = n1, n2, c1, c2
+        else:
+            raise ValueError(kind)
+    return (_store(W1, "bf16"), torch.from_numpy(b1.astype(np.float32)), _store(W2, "bf16"),
+            torch.from_numpy(b2.astype(np.float32)))

@@ -39,6 +39,10 @@ _SIGS = {
     "rehyat_exp2_fma": [_vp, _vp, ctypes.c_int64, _vp],
     "rehyat_forward_ex_workspace_bytes": [_I, _I, _I, _I, _I, _I, _I, _I, ctypes.POINTER(_c_size)],
     "rehyat_forward_ex": [_vp, _vp, _vp, _I, _I, _I, _I, _I, _I, _I, _I, _I, _vp, _vp, _c_size, _vp],
+    "rehyat_phi_mlp": [_vp, _I, _I, _I, _I, _I, _vp, _vp, _vp, _vp, _vp, _vp],
+    "rehyat_forward_phi": [_vp, _vp, _vp, _vp, _vp, _I, _I, _I, _I, _I, _I, _I, _I, _I, _vp, _vp, _c_size, _vp],
+    "rehyat_forward_mlp_workspace_bytes": [_I, _I, _I, _I, _I, _I, _I, _I, ctypes.POINTER(_c_size)],
+    "rehyat_forward_mlp": [_vp] * 11 + [_I] * 9 + [_vp, _vp, _c_size, _vp],
 }
 _RESTYPES = {"rehyat_status_string": ctypes.c_char_p}
 
@@ -158,6 +162,90 @@ def forward_sets(q, k, v, F, S_tok, chunk_frames, overlap_frames, sets="causal",
     ws = alloc_workspace(n.value, q.device) if workspace is None else workspace
     _check(lib().rehyat_forward_ex(_p(q), _p(k), _p(v), B, H, F, S_tok, d, chunk_frames, overlap_frames, SETS[sets],
                                    LAYOUTS[layout], _p(out), _p(ws), ws.numel(), _stream()), "rehyat_forward_ex")
+    return out
+
+
+def _dims(q, F, S_tok, layout):
+    if layout == "bhnd":
+        return _shape(q, F, S_tok)
+    B, N, H, d = q.shape
+    if N != F * S_tok:
+        raise ValueError(f"N={N} != F*S_tok={F * S_tok}")
+    return B, H, N, d
+
+
+def _need_mlp(w, H, d, name):
+    """w = (W1 [H,2d,d] bf16, b1 [H,2d] fp32, W2 [H,2d,2d] bf16, b2 [H,2d] fp32)."""
+    if len(w) != 4:
+        raise ValueError(f"{name} must be (W1, b1, W2, b2)")
+    W1, b1, W2, b2 = w
+    for n, t, dt, shape in (("W1", W1, torch.bfloat16, (H, 2 * d, d)), ("b1", b1, torch.float32, (H, 2 * d)),
+                            ("W2", W2, torch.bfloat16, (H, 2 * d, 2 * d)), ("b2", b2, torch.float32, (H, 2 * d))):
+        _need(t, dt, f"{name}.{n}", len(shape))
+        if tuple(t.shape) != shape:
+            raise ValueError(f"{name}.{n} must be {shape}, got {tuple(t.shape)}")
+    return W1, b1, W2, b2
+
+
+def phi_mlp(x, W1, b1, W2, b2, layout="bhnd", out=None):
+    """rehyat_phi_mlp: learned feature map of x ([B,H,N,d] or [B,N,H,d] bf16)
+    with per-head weights -> phi [B,H,N,2d] bf16."""
+    _need(x, torch.bfloat16, "x")
+    if layout == "bhnd":
+        B, H, N, d = x.shape
+    else:
+        B, N, H, d = x.shape
+    _need_mlp((W1, b1, W2, b2), H, d, "weights")
+    out = torch.empty((B, H, N, 2 * d), dtype=torch.bfloat16, device=x.device) if out is None else out
+    _need(out, torch.bfloat16, "out")
+    _check(lib().rehyat_phi_mlp(_p(x), B, H, N, d, LAYOUTS[layout], _p(W1), _p(b1), _p(W2), _p(b2), _p(out),
+                                _stream()), "rehyat_phi_mlp")
+    return out
+
+
+def forward_phi(q, k, v, phi_q, phi_k, F, S_tok, chunk_frames, overlap_frames, sets="causal", layout="bhnd",
+                out=None, workspace=None):
+    """rehyat_forward_phi: the forward with precomputed feature maps phi_q,
+    phi_k ([B,H,N,2d] bf16, non-negative) in the linear term and states."""
+    for n, t in (("q", q), ("k", k), ("v", v), ("phi_q", phi_q), ("phi_k", phi_k)):
+        _need(t, torch.bfloat16, n)
+    B, H, N, d = _dims(q, F, S_tok, layout)
+    for n, t in (("phi_q", phi_q), ("phi_k", phi_k)):
+        if tuple(t.shape) != (B, H, N, 2 * d):
+            raise ValueError(f"{n} must be {(B, H, N, 2 * d)}")
+    out = torch.empty_like(q) if out is None else out
+    n = _c_size(0)
+    _check(lib().rehyat_forward_ex_workspace_bytes(B, H, F, S_tok, d, chunk_frames, overlap_frames, SETS[sets],
+                                                   ctypes.byref(n)), "rehyat_forward_ex_workspace_bytes")
+    ws = alloc_workspace(n.value, q.device) if workspace is None else workspace
+    _check(lib().rehyat_forward_phi(_p(q), _p(k), _p(v), _p(phi_q), _p(phi_k), B, H, F, S_tok, d, chunk_frames,
+                                    overlap_frames, SETS[sets], LAYOUTS[layout], _p(out), _p(ws), ws.numel(),
+                                    _stream()), "rehyat_forward_phi")
+    return out
+
+
+def forward_mlp_workspace_bytes(B, H, F, S_tok, d, chunk_frames, overlap_frames, sets="causal") -> int:
+    n = _c_size(0)
+    _check(lib().rehyat_forward_mlp_workspace_bytes(B, H, F, S_tok, d, chunk_frames, overlap_frames, SETS[sets],
+                                                    ctypes.byref(n)), "rehyat_forward_mlp_workspace_bytes")
+    return n.value
+
+
+def forward_mlp(q, k, v, wq, wk, F, S_tok, chunk_frames, overlap_frames, sets="causal", layout="bhnd", out=None,
+                workspace=None):
+    """rehyat_forward_mlp: learned phi_q (weights wq) and phi_k (wk), each
+    (W1, b1, W2, b2), then the hybrid forward."""
+    for n, t in (("q", q), ("k", k), ("v", v)):
+        _need(t, torch.bfloat16, n)
+    B, H, N, d = _dims(q, F, S_tok, layout)
+    Wq1, bq1, Wq2, bq2 = _need_mlp(wq, H, d, "wq")
+    Wk1, bk1, Wk2, bk2 = _need_mlp(wk, H, d, "wk")
+    out = torch.empty_like(q) if out is None else out
+    nb = forward_mlp_workspace_bytes(B, H, F, S_tok, d, chunk_frames, overlap_frames, sets)
+    ws = alloc_workspace(nb, q.device) if workspace is None else workspace
+    _check(lib().rehyat_forward_mlp(_p(q), _p(k), _p(v), _p(Wq1), _p(bq1), _p(Wq2), _p(bq2), _p(Wk1), _p(bk1),
+                                    _p(Wk2), _p(bk2), B, H, F, S_tok, d, chunk_frames, overlap_frames, SETS[sets],
+                                    LAYOUTS[layout], _p(out), _p(ws), ws.numel(), _stream()), "rehyat_forward_mlp")
     return out
 
 

@@ -134,3 +134,39 @@ def test_step_frames_cover_the_video():
             folded += ef
             t += 1
         assert folded <= F
+
+
+def test_mlp_validation(lib):
+    def m(**kw):
+        a = dict(x=16, N=100, d=128, layout=0, W1=16, b1=16, W2=16, b2=16, phi=16)
+        a.update(kw)
+        return lib.rehyat_phi_mlp(a["x"], 1, 2, a["N"], a["d"], a["layout"], a["W1"], a["b1"], a["W2"], a["b2"],
+                                  a["phi"], None)
+    assert m(x=0) == R.EINVAL
+    assert m(W2=8) == R.EINVAL           # misaligned weights
+    assert m(b1=0) == R.EINVAL
+    assert m(phi=0) == R.EINVAL
+    assert m(d=96) == R.EUNSUPPORTED
+    assert m(N=0) == R.EINVAL
+    assert m(layout=3) == R.EINVAL
+
+    def fp(phi_q=16, phi_k=16, sets=0, ws=0, nb=0):
+        return lib.rehyat_forward_phi(16, 16, 16, phi_q, phi_k, 1, 1, 4, 8, 64, 2, 1, sets, 0, 16, ws, nb, None)
+    assert fp(phi_q=0) == R.EINVAL
+    assert fp(phi_k=24) == R.EINVAL
+    assert fp(sets=2) == R.EINVAL
+    assert fp(ws=256, nb=1) == R.ENOMEM
+
+    def fm(wk2=16, ws=0, nb=0, d=64):
+        return lib.rehyat_forward_mlp(16, 16, 16, 16, 16, 16, 16, 16, 16, wk2, 16, 1, 1, 4, 8, d, 2, 1, 0, 0, 16,
+                                      ws, nb, None)
+    assert fm(wk2=0) == R.EINVAL
+    assert fm(d=32) == R.EUNSUPPORTED
+    assert fm(ws=256, nb=1) == R.ENOMEM
+
+
+def test_mlp_workspace_holds_both_feature_maps():
+    ex = ctypes.c_size_t(0)
+    R.lib().rehyat_forward_ex_workspace_bytes(1, 12, 21, 1560, 128, 3, 1, 0, ctypes.byref(ex))
+    phi = 12 * 21 * 1560 * 256 * 2            # [B, H, N, 2d] bf16, a multiple of 256 here
+    assert R.forward_mlp_workspace_bytes(1, 12, 21, 1560, 128, 3, 1) == ex.value + 2 * phi

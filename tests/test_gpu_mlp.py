@@ -1,0 +1,202 @@
+"""GPU parity of the learned feature map (two-layer MLP, degree-2 features)
+and of the hybrid forward that uses it, against the fp64 oracle.
+
+The feature-map kernel is checked element by element against a bound derived
+from its arithmetic (below); the forwards use the bf16 tolerances of the
+other parity tests (relative L2 <= 1e-2, max |error| <= 3e-2 RMS).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle.rehyat_oracle as orc
+from linear_attention_video_chunk_b200 import inputs
+from linear_attention_video_chunk_b200 import rehyat as R
+from test_gpu_parity import assert_bf16_close, few_rows, np64
+
+pytestmark = pytest.mark.gpu
+
+U_BF16 = 2.0 ** -8  # unit roundoff of bf16 (8-bit significand)
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    R.lib()
+    yield
+    assert R.device_status() == R.OK, "a device-side wait timed out"
+
+
+def _w64(w):
+    return tuple(t.double().numpy() for t in w)
+
+
+def _oracle_phi(x, w):
+    """fp64 oracle features of x [B,H,N,d] with per-head weights -> [B,H,N,2d]."""
+    W1, b1, W2, b2 = _w64(w)
+    x = np.asarray(x.double().numpy() if isinstance(x, torch.Tensor) else x)
+    return np.stack([np.stack([orc.phi_mlp(x[b, h], W1[h], b1[h], W2[h], b2[h]) for h in range(x.shape[1])])
+                     for b in range(x.shape[0])])
+
+
+def _bound(x, w, ref):
+    """Elementwise error bound of the kernel's arithmetic.  The hidden units
+    relu(W1 x + b1) are rounded to bf16 (relative error <= u = 2^-8) before
+    the second GEMM, so |du_o| <= E_o = u * sum_j |W2[o,j]| |h_j|; 1 + elu is
+    1-Lipschitz, and (psi^2)' = 2 psi; the output is rounded to bf16 once more
+    (<= u |phi|).  fp32 accumulation and the fp32 exp add far less than the
+    25% margin."""
+    W1, b1, W2, b2 = _w64(w)
+    x = x.double().numpy()
+    B, H, N, d = x.shape
+    tol = np.empty_like(ref)
+    for b in range(B):
+        for h in range(H):
+            hid = np.maximum(x[b, h] @ W1[h].T + b1[h], 0.0)
+            E = U_BF16 * (hid @ np.abs(W2[h]).T)
+            psi2 = np.sqrt(ref[b, h, :, d:])
+            tol[b, h, :, :d] = U_BF16 * ref[b, h, :, :d] + E[:, :d]
+            tol[b, h, :, d:] = U_BF16 * ref[b, h, :, d:] + 2.0 * psi2 * E[:, d:] + E[:, d:] ** 2
+    return 1.25 * tol + 1e-6
+
+
+MLP_CASES = [
+    # B, H, N, d, layout, kind, seed
+    (2, 3, 300, 128, "bhnd", "near_identity", 1),   # ragged last tile (300 = 2 x 128 + 44)
+    (1, 2, 1000, 128, "bnhd", "random", 2),         # [B, N, H, d] input
+    (2, 2, 257, 64, "bhnd", "random", 3),           # d = 64, one-row last tile
+    (1, 1, 128, 64, "bnhd", "near_identity", 4),    # exactly one tile
+    (1, 1, 5, 128, "bhnd", "random", 5),            # fewer rows than a tile
+]
+
+
+@pytest.mark.parametrize("B,H,N,d,layout,kind,seed", MLP_CASES)
+def test_phi_mlp_kernel_matches_oracle(B, H, N, d, layout, kind, seed):
+    x = inputs.make_qkv(B, H, N, d, seed, rms_qk=True)[0]
+    w = inputs.make_mlp_weights(H, d, seed, "q", kind)
+    xin = x.transpose(1, 2).contiguous() if layout == "bnhd" else x
+    y = R.phi_mlp(xin.cuda(), *(t.cuda() for t in w), layout=layout)
+    torch.cuda.synchronize()
+    ref = _oracle_phi(x, w)
+    got = np64(y)
+    assert (got >= 0).all()
+    err = np.abs(got - ref)
+    tol = _bound(x, w, ref)
+    bad = err > tol
+    assert not bad.any(), f"{bad.sum()} of {bad.size} features outside the bound; worst {(err / tol).max():.3f}"
+
+
+def test_phi_mlp_identity_weights_give_fixed_phi():
+    """W1 = [I; -I], W2 = [[I, -I]; [I, -I]], zero biases: every step is exact
+    up to the final bf16 rounding, so the kernel returns the fixed phi of the
+    bf16 inputs rounded to bf16 (the oracle's phi, cast by torch)."""
+    B, H, N, d = 1, 2, 200, 128
+    x = inputs.make_qkv(B, H, N, d, 9, rms_qk=True)[0]
+    W1, b1, W2, b2 = orc.mlp_identity_weights(d)
+    w = (torch.from_numpy(np.stack([W1] * H)).to(torch.bfloat16), torch.from_numpy(np.stack([b1] * H)).float(),
+         torch.from_numpy(np.stack([W2] * H)).to(torch.bfloat16), torch.from_numpy(np.stack([b2] * H)).float())
+    y = R.phi_mlp(x.cuda(), *(t.cuda() for t in w)).cpu()
+    ref = torch.from_numpy(orc.phi(x.double().numpy())).to(torch.bfloat16)
+    diff = (y.double() - ref.double()).abs()
+    # psi is computed in fp32 (exp within a few ulp), then rounded: at most one bf16 ulp apart
+    assert (diff <= 2.0 ** -7 * ref.double().abs() + 1e-30).all()
+
+
+PHI_CASES = [
+    # B, H, d, F, S_tok, Tc, To, sets, seed
+    (1, 2, 128, 5, 200, 2, 1, "causal", 40),
+    (1, 2, 64, 5, 200, 2, 1, "causal", 41),
+    (2, 1, 128, 6, 70, 2, 3, "causal", 42),
+    (1, 2, 128, 5, 200, 2, 1, "bidirectional", 43),
+    (1, 1, 128, 3, 150, 4, 1, "causal", 44),        # one chunk: no linear set
+]
+
+
+def _bf16_features(x, w):
+    return torch.from_numpy(_oracle_phi(x, w)).to(torch.bfloat16)
+
+
+@pytest.mark.parametrize("B,H,d,F,S,Tc,To,sets,seed", PHI_CASES)
+def test_forward_phi_matches_oracle(B, H, d, F, S, Tc, To, sets, seed):
+    """Precomputed bf16 features (the oracle's MLP of the bf16 inputs, cast to
+    bf16) fed to both sides."""
+    q, k, v = inputs.make_qkv(B, H, F * S, d, seed, rms_qk=True)
+    Pq = _bf16_features(q, inputs.make_mlp_weights(H, d, seed, "q"))
+    Pk = _bf16_features(k, inputs.make_mlp_weights(H, d, seed, "k"))
+    y = R.forward_phi(q.cuda(), k.cuda(), v.cuda(), Pq.cuda(), Pk.cuda(), F, S, Tc, To, sets=sets)
+    mode = "causal" if sets == "causal" else "bidirectional"
+    ref = orc.oracle_forward(q, k, v, F, S, Tc, To, mode=mode, phi_q=Pq.double().numpy(), phi_k=Pk.double().numpy())
+    assert_bf16_close(np64(y), ref, f"forward_phi {sets}")
+
+
+@pytest.mark.parametrize("layout", ["bhnd", "bnhd"])
+def test_forward_mlp_is_phi_mlp_then_forward_phi(layout):
+    """rehyat_forward_mlp == rehyat_phi_mlp of q and of k, then
+    rehyat_forward_phi: bit for bit (the same kernels in the same order)."""
+    B, H, d, F, S, Tc, To = 1, 2, 128, 6, 130, 3, 1
+    q, k, v = (x.cuda() for x in inputs.make_qkv(B, H, F * S, d, 45, rms_qk=True))
+    wq = tuple(t.cuda() for t in inputs.make_mlp_weights(H, d, 45, "q", "random"))
+    wk = tuple(t.cuda() for t in inputs.make_mlp_weights(H, d, 45, "k", "random"))
+    if layout == "bnhd":
+        q, k, v = (x.transpose(1, 2).contiguous() for x in (q, k, v))
+    y = R.forward_mlp(q, k, v, wq, wk, F, S, Tc, To, layout=layout)
+    Pq = R.phi_mlp(q, *wq, layout=layout)
+    Pk = R.phi_mlp(k, *wk, layout=layout)
+    assert torch.equal(y, R.forward_phi(q, k, v, Pq, Pk, F, S, Tc, To, layout=layout))
+
+
+MLP_FWD_CASES = [
+    # B, H, d, F, S_tok, Tc, To, sets, kind, seed
+    (1, 2, 128, 5, 200, 2, 1, "causal", "near_identity", 50),
+    (1, 2, 64, 7, 90, 2, 3, "causal", "random", 51),
+    (2, 1, 128, 6, 100, 3, 0, "bidirectional", "near_identity", 52),
+]
+
+
+@pytest.mark.parametrize("B,H,d,F,S,Tc,To,sets,kind,seed", MLP_FWD_CASES)
+def test_forward_mlp_matches_oracle(B, H, d, F, S, Tc, To, sets, kind, seed):
+    """End to end against the oracle's fp64 MLP features (no bf16 features on
+    the oracle side)."""
+    q, k, v = inputs.make_qkv(B, H, F * S, d, seed, rms_qk=True)
+    wq = inputs.make_mlp_weights(H, d, seed, "q", kind)
+    wk = inputs.make_mlp_weights(H, d, seed, "k", kind)
+    y = R.forward_mlp(q.cuda(), k.cuda(), v.cuda(), tuple(t.cuda() for t in wq), tuple(t.cuda() for t in wk),
+                      F, S, Tc, To, sets=sets)
+    mode = "causal" if sets == "causal" else "bidirectional"
+    ref = orc.oracle_forward(q, k, v, F, S, Tc, To, mode=mode, phi_q=_oracle_phi(q, wq), phi_k=_oracle_phi(k, wk))
+    assert_bf16_close(np64(y), ref, f"forward_mlp {sets} {kind}")
+
+
+def test_wan13b_480p_forward_mlp_sampled_rows():
+    """The learned-map forward at the Wan2.1-1.3B 480p shape (B=1, H=12,
+    d=128, 21 x 1560 tokens, T_c=3, T_o=1), sampled rows of every head."""
+    B, H, d, F, S, Tc, To = 1, 12, 128, 21, 1560, 3, 1
+    q, k, v = inputs.make_qkv(B, H, F * S, d, 1, rms_qk=True)
+    wq = inputs.make_mlp_weights(H, d, 1, "q")
+    wk = inputs.make_mlp_weights(H, d, 1, "k")
+    y = R.forward_mlp(q.cuda(), k.cuda(), v.cuda(), tuple(t.cuda() for t in wq), tuple(t.cuda() for t in wk),
+                      F, S, Tc, To).cpu()
+    rows = few_rows(F, S, Tc)
+    Pq = _oracle_phi(q, wq)[:, :, rows]
+    Pk = _oracle_phi(k, wk)
+    # the oracle indexes query features by row: give it a full-size array
+    Pq_full = np.zeros(Pk.shape)
+    Pq_full[:, :, rows] = Pq
+    ref = orc.oracle_forward(q, k, v, F, S, Tc, To, rows=rows, phi_q=Pq_full, phi_k=Pk)
+    assert_bf16_close(np64(y[:, :, rows]), ref, "wan13b forward_mlp")
+
+
+def test_forward_mlp_identity_weights_close_to_fixed_phi():
+    """Identity weights make the learned map the fixed phi; the only change is
+    that phi(q) is rounded to bf16 before its exp(-M) scaling."""
+    B, H, d, F, S, Tc, To = 1, 2, 128, 6, 130, 3, 1
+    q, k, v = (x.cuda() for x in inputs.make_qkv(B, H, F * S, d, 46, rms_qk=True))
+    W1, b1, W2, b2 = orc.mlp_identity_weights(d)
+    w = (torch.from_numpy(np.stack([W1] * H)).to(torch.bfloat16).cuda(),
+         torch.from_numpy(np.stack([b1] * H)).float().cuda(),
+         torch.from_numpy(np.stack([W2] * H)).to(torch.bfloat16).cuda(),
+         torch.from_numpy(np.stack([b2] * H)).float().cuda())
+    y = R.forward_mlp(q, k, v, w, w, F, S, Tc, To)
+    ref = R.forward(q, k, v, F, S, Tc, To)
+    assert_bf16_close(np64(y), np64(ref), "identity weights vs fixed phi")
