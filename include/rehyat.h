@@ -182,6 +182,21 @@ int rehyat_forward_mlp(const void* q, const void* k, const void* v,
                        int chunk_frames, int overlap_frames, int sets, int layout,
                        void* out, void* workspace, size_t workspace_bytes, void* stream);
 
+/* rehyat_step with precomputed feature maps (e.g. rehyat_phi_mlp of the
+ * chunk's q and of its window's k): phi_q_c [B, H, Lq, 2d] bf16 replaces the
+ * fixed phi of q_c in the linear term, phi_k_c [B, H, Lk, 2d] bf16 that of
+ * k_c when the first evict_frames * S_tok window keys are folded into the
+ * state (only those rows are read).  Other arguments, the state update and
+ * the frame bookkeeping as rehyat_step; workspace may be NULL (stream-ordered
+ * scratch), else it holds rehyat_step_workspace_bytes(...) bytes, 256-byte
+ * aligned. */
+int rehyat_step_phi(const void* q_c, const void* k_c, const void* v_c,
+                    const void* phi_q_c, const void* phi_k_c,
+                    float* state_S, float* state_z, void* out_c,
+                    int B, int H, int S_tok, int d,
+                    int q_frames, int ctx_frames, int evict_frames,
+                    void* workspace, size_t workspace_bytes, void* stream);
+
 /* fp32 forward (SIMT fp32 throughout, accurate exp); same sets and layout.
  * Meant for small problems and tight-tolerance checks; any size is legal. */
 int rehyat_forward_f32(const float* q, const float* k, const float* v,

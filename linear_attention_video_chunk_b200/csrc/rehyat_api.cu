@@ -251,6 +251,21 @@ bool make_map4(CUtensorMap* m, const void* base, long long inner, long long rows
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// bf16 [depth, rows, inner] written by TMA tile stores: boxes of 32 x 128,
+// 64-byte swizzle (the staging layout of the feature-map kernel).
+bool make_store_map(CUtensorMap* m, void* base, long long inner, long long rows, long long depth) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(rows),
+                        static_cast<cuuint64_t>(depth)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(inner) * 2, static_cast<cuuint64_t>(inner) * 2 * rows};
+  cuuint32_t box[3] = {32u, 128u, 1u};
+  cuuint32_t estr[3] = {1u, 1u, 1u};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 int cuda_status(cudaError_t e) { return e == cudaSuccess ? REHYAT_OK : REHYAT_ECUDA; }
 
 #ifdef REHYAT_TRACE
@@ -366,7 +381,8 @@ int run_phi_mlp(const MlpArgs* maps, int n_maps, int B, int H, int N, int d, lon
   for (int i = 0; i < n_maps; ++i) {
     if (!make_map4(&mp.tm_x[i], maps[i].x, d, N, H, B, rs, hs, bs, 128) ||
         !make_map(&mp.tm_w1[i], maps[i].W1, d, D2, H, static_cast<int>(D2)) ||
-        !make_map(&mp.tm_w2[i], maps[i].W2, D2, D2, H, static_cast<int>(D2)))
+        !make_map(&mp.tm_w2[i], maps[i].W2, D2, D2, H, static_cast<int>(D2)) ||
+        !make_store_map(&mp.tm_phi[i], maps[i].phi, D2, N, static_cast<long long>(B) * H))
       return REHYAT_ECUDA;
     mp.b1[i] = maps[i].b1;
     mp.b2[i] = maps[i].b2;
@@ -383,6 +399,9 @@ int run_phi_mlp(const MlpArgs* maps, int n_maps, int B, int H, int N, int d, lon
   groups = groups < 1 ? 1 : (groups > ntiles ? ntiles : groups);
   if (static_cast<long long>(pairs) * groups > INT_MAX) return REHYAT_EINVAL;
   mp.groups = groups;
+#ifdef REHYAT_TRACE
+  mp.trace = g_trace;
+#endif
   return cuda_status(launch_phi_mlp(d, mp, n_maps, s));
 }
 
@@ -707,25 +726,20 @@ REHYAT_API int rehyat_step_workspace_bytes(int B, int H, int S_tok, int d, int q
   return REHYAT_OK;
 }
 
-REHYAT_API int rehyat_step_ws(const void* q_c, const void* k_c, const void* v_c, float* state_S, float* state_z,
-                              void* out_c, int B, int H, int S_tok, int d, int q_frames, int ctx_frames,
-                              int evict_frames, void* workspace, size_t workspace_bytes, void* stream) {
-  StepPlan P;
-  int st = plan_step(B, H, S_tok, d, q_frames, ctx_frames, evict_frames, &P);
-  if (st != REHYAT_OK) return st;
-  if (check_qkvo(q_c, k_c, v_c, out_c) || check_ptr(state_S) || check_ptr(state_z) || check_ptr(workspace))
-    return REHYAT_EINVAL;
-  if (reinterpret_cast<uintptr_t>(workspace) % 256 != 0) return REHYAT_EINVAL;
-  if (workspace_bytes < P.bytes) return REHYAT_ENOMEM;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  uint8_t* w = static_cast<uint8_t*>(workspace);
+namespace {
+// One step of the recurrent form: split the carried state into bf16 hi/lo,
+// the fused attention of the chunk, then fold the evicted keys into the
+// state.  phi_q / phi_k (optional): precomputed features of the chunk's
+// queries and of the window's keys ([B, H, Lq, 2d], [B, H, Lk, 2d]).
+int run_step(const void* q_c, const void* k_c, const void* v_c, const void* phi_q, const void* phi_k, float* state_S,
+             float* state_z, void* out_c, const StepPlan& P, uint8_t* w, cudaStream_t s) {
   __nv_bfloat16* hi = reinterpret_cast<__nv_bfloat16*>(w + P.off_hi);
   __nv_bfloat16* lo = reinterpret_cast<__nv_bfloat16*>(w + P.off_lo);
-  st = cuda_status(launch_state_split(state_S, static_cast<long long>(P.BH) * 2 * P.D * P.D, hi, lo, s));
+  int st = cuda_status(launch_state_split(state_S, static_cast<long long>(P.BH) * 2 * P.D * P.D, hi, lo, s));
   if (st != REHYAT_OK) return st;
   AttnParams ap;
   std::memset(&ap, 0, sizeof(ap));
-  const long long d_ = P.D, H_ = P.H, Nq_ = P.Nq, Nk_ = P.Nk;
+  const long long d_ = P.D, H_ = P.H, Nq_ = P.Nq, Nk_ = P.Nk, D2 = 2LL * P.D;
   if (!make_map4(&ap.tm_q, q_c, P.D, P.Nq, P.H, P.B, d_, Nq_ * d_, H_ * Nq_ * d_, 128) ||
       !make_map4(&ap.tm_k, k_c, P.D, P.Nk, P.H, P.B, d_, Nk_ * d_, H_ * Nk_ * d_, 128) ||
       !make_map4(&ap.tm_v, v_c, P.D, P.Nk, P.H, P.B, d_, Nk_ * d_, H_ * Nk_ * d_, 128) ||
@@ -744,11 +758,17 @@ REHYAT_API int rehyat_step_ws(const void* q_c, const void* k_c, const void* v_c,
   ap.z_bh = 2LL * P.D;
   ap.z_t = 0;
   ap.out = static_cast<__nv_bfloat16*>(out_c);
-  st = cuda_status(launch_attention(P.D, false, ap, P.n_units, s));
+  if (phi_q != nullptr) {
+    ap.phi_q = static_cast<const __nv_bfloat16*>(phi_q);
+    st = cuda_status(launch_attention_phi(P.D, ap, P.n_units, s));
+  } else {
+    st = cuda_status(launch_attention(P.D, false, ap, P.n_units, s));
+  }
   if (st != REHYAT_OK || P.evict_tok == 0) return st;
   StateParams sp;
   std::memset(&sp, 0, sizeof(sp));
-  if (!make_map4(&sp.tm_k, k_c, P.D, P.Nk, P.H, P.B, d_, Nk_ * d_, H_ * Nk_ * d_, 64) ||
+  if ((phi_k == nullptr && !make_map4(&sp.tm_k, k_c, P.D, P.Nk, P.H, P.B, d_, Nk_ * d_, H_ * Nk_ * d_, 64)) ||
+      (phi_k != nullptr && !make_map4(&sp.tm_phik, phi_k, D2, P.Nk, P.H, P.B, D2, Nk_ * D2, H_ * Nk_ * D2, 64)) ||
       !make_map4(&sp.tm_v, v_c, P.D, P.Nk, P.H, P.B, d_, Nk_ * d_, H_ * Nk_ * d_, 64))
     return REHYAT_ECUDA;
   sp.sg = SegGeom{P.Nk, 0, 0, 1, P.nsplit, 1, P.evict_tok};
@@ -756,9 +776,48 @@ REHYAT_API int rehyat_step_ws(const void* q_c, const void* k_c, const void* v_c,
   sp.H = P.H;
   sp.part_S = reinterpret_cast<float*>(w + P.off_pS);
   sp.part_z = reinterpret_cast<float*>(w + P.off_pz);
-  st = cuda_status(launch_chunk_state(P.D, sp, P.BH * P.nsplit, s));
+  st = cuda_status(phi_k != nullptr ? launch_chunk_state_phi(P.D, sp, P.BH * P.nsplit, s)
+                                    : launch_chunk_state(P.D, sp, P.BH * P.nsplit, s));
   if (st != REHYAT_OK) return st;
   return cuda_status(launch_state_accumulate(sp.part_S, sp.part_z, P.BH, P.nsplit, P.D, state_S, state_z, s));
+}
+}  // namespace
+
+REHYAT_API int rehyat_step_ws(const void* q_c, const void* k_c, const void* v_c, float* state_S, float* state_z,
+                              void* out_c, int B, int H, int S_tok, int d, int q_frames, int ctx_frames,
+                              int evict_frames, void* workspace, size_t workspace_bytes, void* stream) {
+  StepPlan P;
+  int st = plan_step(B, H, S_tok, d, q_frames, ctx_frames, evict_frames, &P);
+  if (st != REHYAT_OK) return st;
+  if (check_qkvo(q_c, k_c, v_c, out_c) || check_ptr(state_S) || check_ptr(state_z) || check_ptr(workspace))
+    return REHYAT_EINVAL;
+  if (reinterpret_cast<uintptr_t>(workspace) % 256 != 0) return REHYAT_EINVAL;
+  if (workspace_bytes < P.bytes) return REHYAT_ENOMEM;
+  return run_step(q_c, k_c, v_c, nullptr, nullptr, state_S, state_z, out_c, P, static_cast<uint8_t*>(workspace),
+                  static_cast<cudaStream_t>(stream));
+}
+
+REHYAT_API int rehyat_step_phi(const void* q_c, const void* k_c, const void* v_c, const void* phi_q_c,
+                               const void* phi_k_c, float* state_S, float* state_z, void* out_c, int B, int H,
+                               int S_tok, int d, int q_frames, int ctx_frames, int evict_frames, void* workspace,
+                               size_t workspace_bytes, void* stream) {
+  StepPlan P;
+  int st = plan_step(B, H, S_tok, d, q_frames, ctx_frames, evict_frames, &P);
+  if (st != REHYAT_OK) return st;
+  if (check_qkvo(q_c, k_c, v_c, out_c) || check_ptr(state_S) || check_ptr(state_z) || check_ptr(phi_q_c) ||
+      check_ptr(phi_k_c))
+    return REHYAT_EINVAL;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  WsGuard own(s);
+  if (workspace == nullptr) {
+    st = own.alloc(P.bytes);
+    if (st != REHYAT_OK) return st;
+    workspace = own.p;
+  } else {
+    if (reinterpret_cast<uintptr_t>(workspace) % 256 != 0) return REHYAT_EINVAL;
+    if (workspace_bytes < P.bytes) return REHYAT_ENOMEM;
+  }
+  return run_step(q_c, k_c, v_c, phi_q_c, phi_k_c, state_S, state_z, out_c, P, static_cast<uint8_t*>(workspace), s);
 }
 
 REHYAT_API int rehyat_step(const void* q_c, const void* k_c, const void* v_c, float* state_S, float* state_z,

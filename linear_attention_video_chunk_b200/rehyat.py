@@ -43,6 +43,7 @@ _SIGS = {
     "rehyat_forward_phi": [_vp, _vp, _vp, _vp, _vp, _I, _I, _I, _I, _I, _I, _I, _I, _I, _vp, _vp, _c_size, _vp],
     "rehyat_forward_mlp_workspace_bytes": [_I, _I, _I, _I, _I, _I, _I, _I, ctypes.POINTER(_c_size)],
     "rehyat_forward_mlp": [_vp] * 11 + [_I] * 9 + [_vp, _vp, _c_size, _vp],
+    "rehyat_step_phi": [_vp] * 8 + [_I] * 7 + [_vp, _c_size, _vp],
 }
 _RESTYPES = {"rehyat_status_string": ctypes.c_char_p}
 
@@ -353,6 +354,27 @@ def step(q_c, k_c, v_c, state_S, state_z, S_tok, q_frames, ctx_frames, evict_fra
     ws = alloc_workspace(nb, q_c.device) if workspace is None else workspace
     _check(lib().rehyat_step_ws(_p(q_c), _p(k_c), _p(v_c), _p(state_S), _p(state_z), _p(out), B, H, S_tok, d,
                                 q_frames, ctx_frames, evict_frames, _p(ws), ws.numel(), _stream()), "rehyat_step_ws")
+    return out
+
+
+def step_phi(q_c, k_c, v_c, phi_q_c, phi_k_c, state_S, state_z, S_tok, q_frames, ctx_frames, evict_frames,
+             out=None, workspace=None):
+    """rehyat_step_phi: one chunk of the recurrent form with precomputed
+    features phi_q_c [B,H,Lq,2d] and phi_k_c [B,H,Lk,2d] (bf16)."""
+    for n, t in (("q_c", q_c), ("k_c", k_c), ("v_c", v_c), ("phi_q_c", phi_q_c), ("phi_k_c", phi_k_c)):
+        _need(t, torch.bfloat16, n)
+    _need(state_S, torch.float32, "state_S")
+    _need(state_z, torch.float32, "state_z", 3)
+    B, H, Lq, d = q_c.shape
+    if Lq != q_frames * S_tok or k_c.shape[2] != (ctx_frames + q_frames) * S_tok:
+        raise ValueError("q_c / k_c lengths do not match the frame counts")
+    if tuple(phi_q_c.shape) != (B, H, Lq, 2 * d) or tuple(phi_k_c.shape) != (B, H, k_c.shape[2], 2 * d):
+        raise ValueError("phi_q_c / phi_k_c must be [B, H, L, 2d] for the chunk's queries / window keys")
+    out = torch.empty_like(q_c) if out is None else out
+    ws = workspace
+    _check(lib().rehyat_step_phi(_p(q_c), _p(k_c), _p(v_c), _p(phi_q_c), _p(phi_k_c), _p(state_S), _p(state_z),
+                                 _p(out), B, H, S_tok, d, q_frames, ctx_frames, evict_frames, _p(ws),
+                                 ws.numel() if ws is not None else 0, _stream()), "rehyat_step_phi")
     return out
 
 

@@ -170,3 +170,16 @@ def test_mlp_workspace_holds_both_feature_maps():
     R.lib().rehyat_forward_ex_workspace_bytes(1, 12, 21, 1560, 128, 3, 1, 0, ctypes.byref(ex))
     phi = 12 * 21 * 1560 * 256 * 2            # [B, H, N, 2d] bf16, a multiple of 256 here
     assert R.forward_mlp_workspace_bytes(1, 12, 21, 1560, 128, 3, 1) == ex.value + 2 * phi
+
+
+def test_step_phi_validation(lib):
+    def sp(**kw):
+        a = dict(q=16, pq=16, pk=16, S=16, ef=1, ws=0, nb=0)
+        a.update(kw)
+        return lib.rehyat_step_phi(a["q"], 16, 16, a["pq"], a["pk"], a["S"], 16, 16, 1, 1, 8, 64, 2, 1, a["ef"],
+                                   a["ws"], a["nb"], None)
+    assert sp(pq=0) == R.EINVAL
+    assert sp(pk=8) == R.EINVAL
+    assert sp(S=0) == R.EINVAL
+    assert sp(ef=4) == R.EINVAL          # evict beyond the window
+    assert sp(ws=256, nb=1) == R.ENOMEM

@@ -200,3 +200,31 @@ def test_forward_mlp_identity_weights_close_to_fixed_phi():
     y = R.forward_mlp(q, k, v, w, w, F, S, Tc, To)
     ref = R.forward(q, k, v, F, S, Tc, To)
     assert_bf16_close(np64(y), np64(ref), "identity weights vs fixed phi")
+
+
+@pytest.mark.parametrize("F,S,Tc,To", [(8, 120, 3, 1), (7, 64, 2, 3), (6, 50, 1, 0)])
+def test_step_phi_streamed_matches_oracle(F, S, Tc, To):
+    """The recurrent form with learned features: chunk by chunk through
+    rehyat_step_phi (features of each chunk's q and window k sliced from the
+    video's), against the oracle (parallel == recurrent with the same bf16
+    features), and against rehyat_forward_phi."""
+    B, H, d = 1, 2, 128
+    q, k, v = inputs.make_qkv(B, H, F * S, d, 71, rms_qk=True)
+    Pq = _bf16_features(q, inputs.make_mlp_weights(H, d, 71, "q", "random"))
+    Pk = _bf16_features(k, inputs.make_mlp_weights(H, d, 71, "k", "random"))
+    qd, kd, vd, Pqd, Pkd = (x.cuda() for x in (q, k, v, Pq, Pk))
+    Sst = torch.zeros(B, H, 2 * d, d, device="cuda")
+    zst = torch.zeros(B, H, 2 * d, device="cuda")
+    outs = []
+    t = 0
+    while t * min(Tc, F) < F:
+        f0, w, cf, qf, ef = R.step_frames(t, F, Tc, To)
+        sl_q, sl_k = slice(f0 * S, (f0 + qf) * S), slice(w * S, (f0 + qf) * S)
+        outs.append(R.step_phi(qd[:, :, sl_q].contiguous(), kd[:, :, sl_k].contiguous(), vd[:, :, sl_k].contiguous(),
+                               Pqd[:, :, sl_q].contiguous(), Pkd[:, :, sl_k].contiguous(), Sst, zst, S, qf, cf, ef))
+        t += 1
+    y = np64(torch.cat(outs, dim=2))
+    ref = orc.oracle_recurrent(q, k, v, F, S, Tc, To, phi_q=Pq.double().numpy(), phi_k=Pk.double().numpy())
+    assert_bf16_close(y, ref, "step_phi vs oracle")
+    yf = np64(R.forward_phi(qd, kd, vd, Pqd, Pkd, F, S, Tc, To))
+    assert np.linalg.norm(y - yf) / np.linalg.norm(yf) <= 5e-3
