@@ -75,7 +75,7 @@ def work(c, sets="causal"):
                 state_bytes=state_bytes, tokens=B * N, mlp_flops=mlp_flops, mlp_bytes=mlp_bytes)
 
 
-KERNEL_SOURCES = ("tc_kernels.cu", "ptx.cuh", "kernels.cuh", "geom.cuh")
+KERNEL_SOURCES = ("tc_kernels.cu", "tc_common.cuh", "ptx.cuh", "kernels.cuh", "geom.cuh")
 TRAFFIC_PROFILE = os.path.join(ROOT, "profiles", "hybrid_chunk_attn_h6_full.md")
 
 

@@ -1,0 +1,334 @@
+// mlp_kernels.cu -- the learned feature map of "ReHyAt: Recurrent Hybrid
+// Attention for Video Diffusion Transformers" (§4.3 Training specification,
+// §7.1 Training Details: a two-layer MLP with degree-2 polynomial features,
+// separate maps for queries and keys), i.e. the §3.2 feature-map equation
+// with P = 2, on the tensor cores (tcgen05 / TMEM / TMA) for sm_100a.
+#include <cstdint>
+
+#include "kernels.cuh"
+#include "ptx.cuh"
+#include "tc_common.cuh"
+
+namespace rehyat {
+namespace {
+
+// ============================================================================
+// Learned feature map: phi = [psi(u_1), psi(u_2)^2], u = W2 relu(W1 x + b1) + b2
+// ============================================================================
+// Two chained GEMMs per 128-row tile, both on the tensor cores with the
+// head's weights resident in shared memory for the CTA's whole life:
+//   H = x W1^T          (SS MMA, M = 128, N = 2D, K = D)    -> TMEM [0, 2D)
+//   R = relu(H + b1)    bf16, written back into TMEM over H's columns
+//   U = R W2^T          (TS MMA, M = 128, N = 2D, K = 2D)   -> TMEM [2D, 4D)
+//   phi = [1 + elu(U_1 + b2_1), (1 + elu(U_2 + b2_2))^2]   bf16 -> global
+// Warps 0-15 run both epilogues: warp w reads TMEM lane quarter w % 4 and
+// column group w / 4 (a quarter of H's and of U's columns); warp 16 is the TMA
+// producer, warp 17 the MMA issuer.  The next H GEMM runs while the epilogue
+// still reads U.  Features leave through shared memory and TMA tile stores
+// (32 features x 128 rows a box, one box per group and chunk step), so each
+// row is written whole instead of 16 bytes per thread at a 2D-element
+// stride; the producer thread issues those stores and waits for them, so the
+// epilogue warps never block on a store.  At D = 128 the weights leave room
+// for one x tile only, and the staging area is that tile once the next H GEMM
+// has read it.
+template <int D>
+struct MlpCfg {
+  static constexpr int HID = 2 * D;                 // hidden width
+  static constexpr int OUT = 2 * D;                 // feature width D'
+  static constexpr int NBX = D / 64;                // 64-column boxes across x and W1
+  static constexpr int NBH = HID / 64;              // ... across the hidden units (W2)
+  static constexpr int XBOX = 128 * 128;            // 128 rows x 128 B
+  static constexpr int X_BYTES = NBX * XBOX;
+  static constexpr int W1BOX = HID * 128;           // HID rows x 128 B
+  static constexpr int W2BOX = OUT * 128;
+  static constexpr int W1_BYTES = NBX * W1BOX;
+  static constexpr int W2_BYTES = NBH * W2BOX;
+  static constexpr int NXB = (D == 128) ? 1 : 2;    // x tile buffers (the weights fill the rest)
+  static constexpr int NG = 4;                      // epilogue column groups
+  static constexpr int HG = HID / NG;               // hidden units of a group
+  static constexpr int OG = OUT / NG;               // features of a group
+  static constexpr int STG_BOX = 128 * 64;          // 32 features x 128 rows, bf16
+  static constexpr int STG_STEP = NG * STG_BOX;     // one chunk step of every group
+  static constexpr bool ALIAS = (D == 128);         // staging = the (single) x tile buffer
+  static constexpr int OFF_W1 = 0;
+  static constexpr int OFF_W2 = W1_BYTES;
+  static constexpr int OFF_X = OFF_W2 + W2_BYTES;
+  static constexpr int OFF_STG = ALIAS ? OFF_X : OFF_X + NXB * X_BYTES;
+  static constexpr int OFF_BAR = ALIAS ? OFF_X + NXB * X_BYTES : OFF_STG + STG_STEP;
+  static constexpr int SMEM = OFF_BAR + 256 + 1024;
+  static constexpr uint32_t TMEM_COLS = (HID + OUT <= 256) ? 256u : 512u;
+  static constexpr int EPI_WARPS = 4 * NG;
+  static constexpr int THREADS = 32 * EPI_WARPS + 64;
+  static constexpr int B_W = 0, B_X = 1, B_XE = 1 + NXB, B_H = 1 + 2 * NXB, B_R = B_H + 1, B_U = B_H + 2,
+                       B_UE = B_H + 3, B_STF = B_H + 4, B_STE = B_H + 5, B_FIN = B_H + 6;
+  static constexpr int NC = OG / 32;                // 32-feature chunk steps of a tile
+  static_assert(!ALIAS || (NXB == 1 && X_BYTES >= STG_STEP), "staging inside the x tile");
+  static_assert(HG % 32 == 0 && OG % 32 == 0, "whole 32-column chunks per group");
+  // both GEMMs: A and B K-major (x rows / R rows by W rows)
+  static constexpr uint32_t IDESC1 = idesc_bf16_f32(128, HID, 0, 0);
+  static constexpr uint32_t IDESC2 = idesc_bf16_f32(128, OUT, 0, 0);
+  static_assert(SMEM <= 232448, "shared memory");
+  static_assert((B_FIN + 1) * 8 <= 128, "barrier area");
+  static_assert(HID + OUT <= 512, "tensor memory");
+};
+
+template <int D>
+__global__ void __launch_bounds__(MlpCfg<D>::THREADS, 1) phi_mlp_kernel(const __grid_constant__ MlpParams p) {
+  using C = MlpCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int grp_id = blockIdx.x % p.groups;  // CTA = (map, bh, row group)
+  const int rest = blockIdx.x / p.groups;
+  const int bh = rest % p.BH;
+  const int m = rest / p.BH;
+  const int hh = bh % p.H, bb = bh / p.H;
+  const int ntiles = cdiv(p.N, 128);
+  const int my_tiles = grp_id < ntiles ? cdiv(ntiles - grp_id, p.groups) : 0;
+  if (my_tiles == 0) return;  // uniform exit, before any barrier or TMEM use
+
+  uint8_t* barea = smem + C::OFF_BAR;
+  const uint32_t bar0 = smem_u32(barea);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(barea + 128);
+  volatile int* abort = reinterpret_cast<volatile int*>(barea + 132);
+#define BAR(i) (bar0 + 8u * static_cast<uint32_t>(i))
+  if (threadIdx.x == 0) {
+    mbar_init(BAR(C::B_W), 1);
+    for (int i = 0; i < C::NXB; ++i) {
+      mbar_init(BAR(C::B_X + i), 1);
+      mbar_init(BAR(C::B_XE + i), 1);
+    }
+    mbar_init(BAR(C::B_H), 1);
+    mbar_init(BAR(C::B_R), C::EPI_WARPS);
+    mbar_init(BAR(C::B_U), 1);
+    mbar_init(BAR(C::B_UE), C::EPI_WARPS);
+    mbar_init(BAR(C::B_STF), C::EPI_WARPS);
+    mbar_init(BAR(C::B_STE), 1);
+    mbar_init(BAR(C::B_FIN), 1);
+    *abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == C::EPI_WARPS && lane == 0) {
+    prefetch_tmap(&p.tm_x[m]);
+    prefetch_tmap(&p.tm_w1[m]);
+    prefetch_tmap(&p.tm_w2[m]);
+    prefetch_tmap(&p.tm_phi[m]);
+  }
+  if (warp == C::EPI_WARPS + 1) {
+    tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp < C::EPI_WARPS) {
+    // ============================ epilogues ============================
+    const int quarter = warp & 3, g = warp >> 2;
+    const uint32_t lane_off = static_cast<uint32_t>(32 * quarter) << 16;
+    const float4* b1 = reinterpret_cast<const float4*>(p.b1[m] + hh * C::HID + g * C::HG);  // group's hidden units
+    const float4* b2 = reinterpret_cast<const float4*>(p.b2[m] + hh * C::OUT + g * C::OG);  // group's features
+    const bool square = g * C::OG >= D;  // features D..2D-1 are psi_2^2
+    const int r = 32 * quarter + lane;   // row inside the tile
+    const uint32_t my_stg = smem_u32(smem + C::OFF_STG) + g * C::STG_BOX + r * 64;
+    const int swz = (r >> 1) & 3;
+    // After a failed wait the remaining waits are skipped and the loop runs
+    // out without blocking.
+    bool ok = true;
+    for (int it = 0; it < my_tiles; ++it) {
+      ok = ok && warp_wait(BAR(C::B_H), it & 1, abort);
+      if (threadIdx.x == 0) TRACE(0, it);
+      tc_fence_after();
+      // R = relu(H + b1) as bf16 pairs: the group's HG hidden units go to the
+      // first HG/2 of its own HG columns (chunk c is read before any column it
+      // overwrites, and the groups' column ranges are disjoint)
+#pragma unroll 1
+      for (int c = 0; c < C::HG / 32; ++c) {
+        uint32_t v[32];
+        tmem_ld32(tmem + lane_off + g * C::HG + 32 * c, v);
+        tmem_ld_wait();
+        reg_fence(v);
+        uint32_t rr[16];
+#pragma unroll
+        for (int q4 = 0; q4 < 8; ++q4) {
+          const float4 bv = __ldg(b1 + 8 * c + q4);
+          rr[2 * q4] = pack_bf16(fmaxf(__uint_as_float(v[4 * q4]) + bv.x, 0.f),
+                                 fmaxf(__uint_as_float(v[4 * q4 + 1]) + bv.y, 0.f));
+          rr[2 * q4 + 1] = pack_bf16(fmaxf(__uint_as_float(v[4 * q4 + 2]) + bv.z, 0.f),
+                                     fmaxf(__uint_as_float(v[4 * q4 + 3]) + bv.w, 0.f));
+        }
+        tmem_st16(tmem + lane_off + g * C::HG + 16 * c, rr);
+      }
+      warp_release(BAR(C::B_R), lane);
+      if (threadIdx.x == 0) TRACE(1, it);
+      ok = ok && warp_wait(BAR(C::B_U), it & 1, abort);
+      if (threadIdx.x == 0) TRACE(2, it);
+      tc_fence_after();
+      // phi = psi(U + b2), squared for the second half, one row a thread,
+      // staged in shared memory (64-byte swizzle: 16-byte chunk j of row r at
+      // chunk j ^ ((r >> 1) & 3)); the producer thread stores each step by TMA
+#pragma unroll 1
+      for (int c = 0; c < C::NC; ++c) {
+        uint32_t v[32];
+        tmem_ld32(tmem + lane_off + C::HID + g * C::OG + 32 * c, v);
+        tmem_ld_wait();
+        reg_fence(v);
+        if (c == C::NC - 1) {  // U fully read: the next tile's second GEMM may overwrite it
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(BAR(C::B_UE));
+        }
+        uint32_t o[16];
+#pragma unroll
+        for (int q4 = 0; q4 < 8; ++q4) {
+          const float4 bv = __ldg(b2 + 8 * c + q4);
+          const float u0 = __uint_as_float(v[4 * q4]) + bv.x, u1 = __uint_as_float(v[4 * q4 + 1]) + bv.y;
+          const float u2 = __uint_as_float(v[4 * q4 + 2]) + bv.z, u3 = __uint_as_float(v[4 * q4 + 3]) + bv.w;
+          float f0 = psi1(u0), f1 = psi1(u1), f2 = psi1(u2), f3 = psi1(u3);
+          if (square) {
+            f0 *= f0;
+            f1 *= f1;
+            f2 *= f2;
+            f3 *= f3;
+          }
+          o[2 * q4] = pack_bf16(f0, f1);
+          o[2 * q4 + 1] = pack_bf16(f2, f3);
+        }
+        if (c == 0 && threadIdx.x == 0) TRACE(3, it);
+        if (c == 0 && C::ALIAS && it + 1 < my_tiles)  // staging = x tile: the next H GEMM has read it
+          ok = ok && warp_wait(BAR(C::B_XE), (it + 1) & 1, abort);
+        const int step = it * C::NC + c;  // staging use; the previous one must have been stored
+        ok = ok && warp_wait(BAR(C::B_STE), (step & 1) ^ 1, abort);
+        if (c == 0 && threadIdx.x == 0) TRACE(4, it);
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(my_stg + ((j ^ swz) << 4)), "r"(o[4 * j]),
+                       "r"(o[4 * j + 1]), "r"(o[4 * j + 2]), "r"(o[4 * j + 3])
+                       : "memory");
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(BAR(C::B_STF));
+      }
+    }
+  } else if (warp == C::EPI_WARPS) {
+    // ================ TMA producer: x tiles in, features out ================
+    if (lane == 0) {
+      mbar_arrive_expect_tx(BAR(C::B_W), C::W1_BYTES + C::W2_BYTES);
+      for (int b = 0; b < C::NBX; ++b)
+        tma_load_3d(smem_u32(smem + C::OFF_W1 + b * C::W1BOX), &p.tm_w1[m], BAR(C::B_W), 64 * b, 0, hh);
+      for (int b = 0; b < C::NBH; ++b)
+        tma_load_3d(smem_u32(smem + C::OFF_W2 + b * C::W2BOX), &p.tm_w2[m], BAR(C::B_W), 64 * b, 0, hh);
+      bool ok = true;
+      int loaded = 0;  // x tiles issued
+      // x tile `it` into its slot once the H GEMM of the slot's previous tile
+      // has read it (aliased: and once the features staged there have been
+      // stored, which program order below guarantees)
+      auto load_x = [&](int it) {
+        const int slot = it % C::NXB;
+        ok = ok && mbar_wait(BAR(C::B_XE + slot), ((it / C::NXB) & 1) ^ 1, abort);
+        if (!ok) return;
+        TRACE(11, it);
+        const uint32_t dst = smem_u32(smem + C::OFF_X + slot * C::X_BYTES);
+        mbar_arrive_expect_tx(BAR(C::B_X + slot), C::X_BYTES);
+        for (int b = 0; b < C::NBX; ++b)
+          tma_load_4d(dst + b * C::XBOX, &p.tm_x[m], BAR(C::B_X + slot), 64 * b, 128 * (grp_id + it * p.groups), hh,
+                      bb);
+        loaded = it + 1;
+      };
+      for (int it = 0; it < my_tiles && it < 2; ++it) load_x(it);
+      for (int it = 0; it < my_tiles && ok; ++it) {
+        for (int c = 0; c < C::NC && ok; ++c) {
+          const int step = it * C::NC + c;
+          ok = mbar_wait(BAR(C::B_STF), step & 1, abort);
+          if (!ok) break;
+          const uint32_t stg0 = smem_u32(smem + C::OFF_STG);
+          for (int gg = 0; gg < C::NG; ++gg)
+            tma_store_3d(&p.tm_phi[m], stg0 + gg * C::STG_BOX, gg * C::OG + 32 * c, 128 * (grp_id + it * p.groups),
+                         bh);
+          bulk_commit();
+          TRACE(5 + (c & 1), it);
+          bulk_wait_read<0>();  // the staging area may be written again
+          mbar_arrive(BAR(C::B_STE));
+        }
+        TRACE(7, it);
+        if (it + 2 < my_tiles) load_x(it + 2);
+      }
+      bulk_wait<0>();  // every feature row written before the CTA exits
+      drain_wait(BAR(C::B_W), 0);
+      for (int i2 = (loaded > C::NXB ? loaded - C::NXB : 0); i2 < loaded; ++i2)
+        drain_wait(BAR(C::B_X + i2 % C::NXB), (i2 / C::NXB) & 1);
+    }
+  } else {
+    // ============================ MMA issuer ============================
+    if (lane == 0) {
+      constexpr uint32_t HI = desc_hi_sw128(1024);  // K-major: 8-row groups 1024 B apart
+      const uint32_t lo_w1 = desc_lo(smem_u32(smem + C::OFF_W1), 16);
+      const uint32_t lo_w2 = desc_lo(smem_u32(smem + C::OFF_W2), 16);
+      bool ok = mbar_wait(BAR(C::B_W), 0, abort);
+      for (int it = 0; it < my_tiles && ok; ++it) {
+        const int slot = it % C::NXB;
+        ok = mbar_wait(BAR(C::B_X + slot), (it / C::NXB) & 1, abort);
+        if (!ok) break;
+        TRACE(8, it);
+        tc_fence_after();
+        const uint32_t lo_x = desc_lo(smem_u32(smem + C::OFF_X + slot * C::X_BYTES), 16);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk)  // K-step kk: box kk/4, 32 B into the swizzled row
+          mma_ss(tmem, desc_join(lo_x + (((kk >> 2) * C::XBOX + (kk & 3) * 32) >> 4), HI),
+                 desc_join(lo_w1 + (((kk >> 2) * C::W1BOX + (kk & 3) * 32) >> 4), HI), C::IDESC1, kk > 0 ? 1u : 0u);
+        mma_commit(BAR(C::B_XE + slot));
+        mma_commit(BAR(C::B_H));
+        TRACE(9, it);
+        // R of this tile written, and U free (the previous tile's features stored)
+        ok = mbar_wait(BAR(C::B_R), it & 1, abort) && mbar_wait(BAR(C::B_UE), (it & 1) ^ 1, abort);
+        if (!ok) break;
+        TRACE(10, it);
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < C::HID / 16; ++kk) {  // 16 hidden units = 8 packed columns of R
+          const uint32_t a = tmem + (kk / (C::HG / 16)) * C::HG + (kk % (C::HG / 16)) * 8;
+          mma_ts(tmem + C::HID, a, desc_join(lo_w2 + (((kk >> 2) * C::W2BOX + (kk & 3) * 32) >> 4), HI), C::IDESC2,
+                 kk > 0 ? 1u : 0u);
+        }
+        mma_commit(BAR(C::B_U));
+      }
+      mma_commit(BAR(C::B_FIN));
+      drain_wait(BAR(C::B_FIN), 0);
+    }
+  }
+#undef BAR
+  tc_fence_before();
+  __syncthreads();
+  if (warp == C::EPI_WARPS + 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+}  // namespace
+
+template <int D>
+static cudaError_t launch_mlp_t(const MlpParams& p, int n_maps, cudaStream_t s) {
+  auto* k = phi_mlp_kernel<D>;
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, MlpCfg<D>::SMEM);
+  if (e != cudaSuccess) return e;
+  k<<<n_maps * p.BH * p.groups, MlpCfg<D>::THREADS, MlpCfg<D>::SMEM, s>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_phi_mlp(int D, const MlpParams& p, int n_maps, cudaStream_t s) {
+  if (p.N <= 0 || n_maps <= 0) return cudaSuccess;
+  return D == 128 ? launch_mlp_t<128>(p, n_maps, s) : launch_mlp_t<64>(p, n_maps, s);
+}
+
+cudaError_t read_and_clear_device_error_mlp(unsigned int* v) {
+  cudaError_t e = cudaMemcpyFromSymbol(v, g_device_error, sizeof(unsigned int));
+  if (e != cudaSuccess) return e;
+  const unsigned int zero = 0;
+  return cudaMemcpyToSymbol(g_device_error, &zero, sizeof(unsigned int));
+}
+
+}  // namespace rehyat

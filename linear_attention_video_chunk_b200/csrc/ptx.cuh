@@ -12,9 +12,10 @@
 
 namespace rehyat {
 
-// Device error word: bit 0 = a bounded wait ran out.  Read and cleared by
-// rehyat_device_status().  (This header is included by one translation unit.)
-__device__ unsigned int g_device_error = 0;
+// Device error word: bit 0 = a bounded wait ran out.  Every translation unit
+// that includes this header has its own word and a reader that
+// rehyat_device_status() calls (read and clear).
+static __device__ unsigned int g_device_error = 0;
 
 constexpr unsigned int kErrTimeout = 1u;
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s
