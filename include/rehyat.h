@@ -197,6 +197,26 @@ int rehyat_step_phi(const void* q_c, const void* k_c, const void* v_c,
                     int q_frames, int ctx_frames, int evict_frames,
                     void* workspace, size_t workspace_bytes, void* stream);
 
+/* rehyat_forward_ex on HOST buffers: copies q, k, v (host, ideally
+ * page-locked) into the device workspace, runs the forward, and copies the
+ * result back into out_host, all enqueued on `stream` (asynchronous for
+ * page-locked host memory: the result is in out_host once the stream has
+ * reached this point; pageable memory makes the copies synchronous).
+ * Keys and values are copied first, so the copy of q can overlap nothing but
+ * is ready before the attention stage.  The workspace (device, 256-byte
+ * aligned, caller-owned, rehyat_forward_host_workspace_bytes(...) bytes)
+ * holds the device copies of q, k, v, out and the forward's scratch; callers
+ * that alternate two workspaces on two streams overlap one call's copies with
+ * another's kernels.  Host tensors in `layout`, [B, H, N, d] or [B, N, H, d]
+ * bf16.  Returns REHYAT_ECUDA if a copy cannot be enqueued. */
+int rehyat_forward_host_workspace_bytes(int B, int H, int F, int S_tok, int d,
+                                        int chunk_frames, int overlap_frames, int sets,
+                                        size_t* bytes);
+int rehyat_forward_host(const void* q_host, const void* k_host, const void* v_host,
+                        int B, int H, int F, int S_tok, int d,
+                        int chunk_frames, int overlap_frames, int sets, int layout,
+                        void* out_host, void* workspace, size_t workspace_bytes, void* stream);
+
 /* fp32 forward (SIMT fp32 throughout, accurate exp); same sets and layout.
  * Meant for small problems and tight-tolerance checks; any size is legal. */
 int rehyat_forward_f32(const float* q, const float* k, const float* v,

@@ -541,6 +541,56 @@ REHYAT_API int rehyat_forward_ex(const void* q, const void* k, const void* v, in
   return run_attention(q, k, v, P, w, out, nullptr, nullptr, nullptr, nullptr, nullptr, s);
 }
 
+namespace {
+// Device copies of q, k, v, out, then the forward's own scratch.
+size_t host_tensor_bytes(const FwdPlan& P) { return align256(static_cast<size_t>(P.BH) * P.N * P.D * 2); }
+}  // namespace
+
+REHYAT_API int rehyat_forward_host_workspace_bytes(int B, int H, int F, int S_tok, int d, int chunk_frames,
+                                                   int overlap_frames, int sets, size_t* bytes) {
+  if (bytes == nullptr) return REHYAT_EINVAL;
+  FwdPlan P;
+  int st = plan_forward_sets(B, H, F, S_tok, d, chunk_frames, overlap_frames, sets, &P);
+  if (st != REHYAT_OK) return st;
+  *bytes = 4 * host_tensor_bytes(P) + P.bytes;
+  return REHYAT_OK;
+}
+
+REHYAT_API int rehyat_forward_host(const void* q_host, const void* k_host, const void* v_host, int B, int H, int F,
+                                   int S_tok, int d, int chunk_frames, int overlap_frames, int sets, int layout,
+                                   void* out_host, void* workspace, size_t workspace_bytes, void* stream) {
+  FwdPlan P;
+  int st = plan_forward_sets(B, H, F, S_tok, d, chunk_frames, overlap_frames, sets, &P);
+  if (st != REHYAT_OK) return st;
+  st = apply_layout(layout, &P);
+  if (st != REHYAT_OK) return st;
+  if (q_host == nullptr || k_host == nullptr || v_host == nullptr || out_host == nullptr || workspace == nullptr)
+    return REHYAT_EINVAL;
+  if (reinterpret_cast<uintptr_t>(workspace) % 256 != 0) return REHYAT_EINVAL;
+  const size_t tb = host_tensor_bytes(P);
+  if (workspace_bytes < 4 * tb + P.bytes) return REHYAT_ENOMEM;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* w = static_cast<uint8_t*>(workspace);
+  uint8_t *qd = w, *kd = w + tb, *vd = w + 2 * tb, *od = w + 3 * tb;
+  const size_t n = static_cast<size_t>(P.BH) * P.N * P.D * 2;  // bytes of one tensor
+  // keys and values first: the states stage needs only them
+  if (cudaMemcpyAsync(kd, k_host, n, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+      cudaMemcpyAsync(vd, v_host, n, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+      cudaMemcpyAsync(qd, q_host, n, cudaMemcpyHostToDevice, s) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return REHYAT_ECUDA;
+  }
+  st = run_states(kd, vd, P, w + 4 * tb, nullptr, nullptr, s);
+  if (st != REHYAT_OK) return st;
+  st = run_attention(qd, kd, vd, P, w + 4 * tb, od, nullptr, nullptr, nullptr, nullptr, nullptr, s);
+  if (st != REHYAT_OK) return st;
+  if (cudaMemcpyAsync(out_host, od, n, cudaMemcpyDeviceToHost, s) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return REHYAT_ECUDA;
+  }
+  return REHYAT_OK;
+}
+
 REHYAT_API int rehyat_phi_mlp(const void* x, int B, int H, int N, int d, int layout, const void* W1,
                               const float* b1, const void* W2, const float* b2, void* phi, void* stream) {
   if (B < 1 || H < 1 || N < 1) return REHYAT_EINVAL;

@@ -44,6 +44,8 @@ _SIGS = {
     "rehyat_forward_mlp_workspace_bytes": [_I, _I, _I, _I, _I, _I, _I, _I, ctypes.POINTER(_c_size)],
     "rehyat_forward_mlp": [_vp] * 11 + [_I] * 9 + [_vp, _vp, _c_size, _vp],
     "rehyat_step_phi": [_vp] * 8 + [_I] * 7 + [_vp, _c_size, _vp],
+    "rehyat_forward_host_workspace_bytes": [_I, _I, _I, _I, _I, _I, _I, _I, ctypes.POINTER(_c_size)],
+    "rehyat_forward_host": [_vp, _vp, _vp] + [_I] * 9 + [_vp, _vp, _c_size, _vp],
 }
 _RESTYPES = {"rehyat_status_string": ctypes.c_char_p}
 
@@ -247,6 +249,30 @@ def forward_mlp(q, k, v, wq, wk, F, S_tok, chunk_frames, overlap_frames, sets="c
     _check(lib().rehyat_forward_mlp(_p(q), _p(k), _p(v), _p(Wq1), _p(bq1), _p(Wq2), _p(bq2), _p(Wk1), _p(bk1),
                                     _p(Wk2), _p(bk2), B, H, F, S_tok, d, chunk_frames, overlap_frames, SETS[sets],
                                     LAYOUTS[layout], _p(out), _p(ws), ws.numel(), _stream()), "rehyat_forward_mlp")
+    return out
+
+
+def forward_host_workspace_bytes(B, H, F, S_tok, d, chunk_frames, overlap_frames, sets="causal") -> int:
+    n = _c_size(0)
+    _check(lib().rehyat_forward_host_workspace_bytes(B, H, F, S_tok, d, chunk_frames, overlap_frames, SETS[sets],
+                                                     ctypes.byref(n)), "rehyat_forward_host_workspace_bytes")
+    return n.value
+
+
+def forward_host(q, k, v, F, S_tok, chunk_frames, overlap_frames, out, workspace, sets="causal", layout="bhnd",
+                 stream=None):
+    """rehyat_forward_host: q, k, v and out are HOST tensors (page-locked for
+    asynchronous copies); workspace is a device uint8 tensor of
+    forward_host_workspace_bytes(...) bytes.  Enqueued on `stream` (default:
+    torch's current stream); synchronise before reading out."""
+    for n_, t in (("q", q), ("k", k), ("v", v), ("out", out)):
+        if not isinstance(t, torch.Tensor) or t.is_cuda or t.dtype != torch.bfloat16 or not t.is_contiguous():
+            raise ValueError(f"{n_} must be a contiguous bf16 host tensor")
+    B, H, N, d = _dims(q, F, S_tok, layout)
+    st = _vp(stream.cuda_stream) if stream is not None else _stream()
+    _check(lib().rehyat_forward_host(_p(q), _p(k), _p(v), B, H, F, S_tok, d, chunk_frames, overlap_frames, SETS[sets],
+                                     LAYOUTS[layout], _p(out), _p(workspace), workspace.numel(), st),
+           "rehyat_forward_host")
     return out
 
 

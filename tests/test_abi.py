@@ -183,3 +183,16 @@ def test_step_phi_validation(lib):
     assert sp(S=0) == R.EINVAL
     assert sp(ef=4) == R.EINVAL          # evict beyond the window
     assert sp(ws=256, nb=1) == R.ENOMEM
+
+
+def test_forward_host_validation(lib):
+    def fh(q=16, ws=256, nb=1 << 40, d=64):
+        return lib.rehyat_forward_host(q, 16, 16, 1, 1, 4, 8, d, 2, 1, 0, 0, 16, ws, nb, None)
+    assert fh(q=0) == R.EINVAL
+    assert fh(ws=0) == R.EINVAL
+    assert fh(ws=272) == R.EINVAL        # misaligned workspace
+    assert fh(nb=1) == R.ENOMEM
+    assert fh(d=96) == R.EUNSUPPORTED
+    ex = ctypes.c_size_t(0)
+    lib.rehyat_forward_ex_workspace_bytes(1, 12, 21, 1560, 128, 3, 1, 0, ctypes.byref(ex))
+    assert R.forward_host_workspace_bytes(1, 12, 21, 1560, 128, 3, 1) == ex.value + 4 * 12 * 32760 * 128 * 2

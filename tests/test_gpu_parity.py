@@ -441,3 +441,24 @@ def test_wan13b_480p_bnhd_sampled_rows():
     rows = few_rows(F, S, Tc)
     ref = orc.oracle_forward(q, k, v, F, S, Tc, To, rows=rows)
     assert_bf16_close(np64(y[:, :, rows]), ref, "bnhd 1.3B")
+
+
+@pytest.mark.parametrize("layout", ["bhnd", "bnhd"])
+def test_forward_host_buffers_equal_device_forward(layout):
+    """rehyat_forward_host (host q/k/v/out, copies inside the call) returns the
+    device forward's result bit for bit, on two streams with two workspaces
+    in flight at once."""
+    B, H, d, F, S, Tc, To = 1, 2, 128, 6, 130, 3, 1
+    q, k, v = inputs.make_qkv(B, H, F * S, d, 140, rms_qk=True, pin=True)
+    if layout == "bnhd":
+        q, k, v = (x.transpose(1, 2).contiguous().pin_memory() for x in (q, k, v))
+    ref = R.forward_sets(q.cuda(), k.cuda(), v.cuda(), F, S, Tc, To, layout=layout).cpu()
+    nb = R.forward_host_workspace_bytes(B, H, F, S, d, Tc, To)
+    streams = [torch.cuda.Stream(), torch.cuda.Stream()]
+    wss = [R.alloc_workspace(nb, "cuda") for _ in range(2)]
+    outs = [torch.empty(q.shape, dtype=torch.bfloat16, pin_memory=True) for _ in range(2)]
+    for i in range(2):
+        R.forward_host(q, k, v, F, S, Tc, To, outs[i], wss[i], layout=layout, stream=streams[i])
+    torch.cuda.synchronize()
+    for o in outs:
+        assert torch.equal(o, ref)
