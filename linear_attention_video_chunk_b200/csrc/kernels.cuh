@@ -51,22 +51,6 @@ struct StateParams {
   float* part_z;      // [BH, n_seg, nsplit, 2D] fp32
 };
 
-// Learned feature map (two-layer MLP, degree-2 polynomial features) on the
-// tensor cores: phi[row] = [psi_1, psi_2^2] of u = W2 relu(W1 x + b1) + b2,
-// psi = 1 + elu.  Up to two maps (phi_q of q, phi_k of k) per launch; one CTA
-// per (map, bh, row group) walks that group's 128-row tiles.
-struct MlpParams {
-  CUtensorMap tm_x[2];    // 4-D {D, N, H, B} bf16, box {64, 128, 1, 1}
-  CUtensorMap tm_w1[2];   // [H, 2D, D] bf16, box {64, 2D, 1}
-  CUtensorMap tm_w2[2];   // [H, 2D, 2D] bf16, box {64, 2D, 1}
-  const float* b1[2];     // [H, 2D]
-  const float* b2[2];     // [H, 2D]
-  __nv_bfloat16* phi[2];  // [BH, N, 2D]
-  CUtensorMap tm_phi[2];  // phi as 3-D {2D, N, BH}, box {32, 128, 1}, 64-byte swizzle (stores)
-  int N, H, BH, groups;
-  unsigned long long* trace;  // clock64 stamps, only with -DREHYAT_TRACE (else unused)
-};
-
 // fp32 SIMT paths
 struct AttnF32Params {
   ChunkGeom g;
@@ -100,7 +84,6 @@ cudaError_t launch_chunk_state(int D, const StateParams& p, int n_ctas, cudaStre
 // states) and phi(Q) rows from p.phi_q (the attention epilogue).
 cudaError_t launch_attention_phi(int D, const AttnParams& p, int n_units, cudaStream_t s);
 cudaError_t launch_chunk_state_phi(int D, const StateParams& p, int n_ctas, cudaStream_t s);
-cudaError_t launch_phi_mlp(int D, const MlpParams& p, int n_maps, cudaStream_t s);
 // Exclusive prefix over segments (and sum over pieces): writes the state
 // entering each chunk, either as bf16 hi/lo (hi, lo non-null) or fp32 (Sf).
 cudaError_t launch_state_scan(const float* part_S, const float* part_z, int BH, int n_seg,

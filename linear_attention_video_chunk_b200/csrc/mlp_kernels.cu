@@ -5,7 +5,8 @@
 // with P = 2, on the tensor cores (tcgen05 / TMEM / TMA) for sm_100a.
 #include <cstdint>
 
-#include "kernels.cuh"
+#include "geom.cuh"
+#include "mlp.cuh"
 #include "ptx.cuh"
 #include "tc_common.cuh"
 

@@ -8,6 +8,7 @@
 
 #include "geom.cuh"
 #include "kernels.cuh"
+#include "mlp.cuh"
 #include "rehyat.h"
 
 #define REHYAT_API extern "C" __attribute__((visibility("default")))
