@@ -179,10 +179,17 @@ def oracle_sample_rate(c, q, k, v, budget_s):
     N = c["F"] * c["S_tok"]
     rng = np.random.default_rng(7)
     args = (c["F"], c["S_tok"], c["T_c"], c["T_o"])
+    # two calibration samples separate the per-call cost (phi of every key)
+    # from the per-row cost, so the measured sample lasts about budget_s
     t0 = time.perf_counter()
     orc.oracle_forward(q, k, v, *args, rows=np.sort(rng.choice(N, 8, replace=False)))
     t8 = time.perf_counter() - t0
-    n = int(max(8, min(N, 8 * budget_s / max(t8, 1e-3))))
+    t0 = time.perf_counter()
+    orc.oracle_forward(q, k, v, *args, rows=np.sort(rng.choice(N, 64, replace=False)))
+    t64 = time.perf_counter() - t0
+    per_row = max((t64 - t8) / 56, 1e-6)
+    fixed = max(t8 - 8 * per_row, 0.0)
+    n = int(max(8, min(N, (budget_s - fixed) / per_row)))
     rows = np.sort(rng.choice(N, n, replace=False))
     t0 = time.perf_counter()
     orc.oracle_forward(q, k, v, *args, rows=rows)
@@ -599,11 +606,17 @@ def run_reference(args):
     N = F * S
     rng = np.random.default_rng(11)
     per_step_budget = max(0.2, 150.0 / max(1, args.steps + args.warmup))
-    # size each step's row sample from a calibration call
+    # size each step's row sample from two calibration calls (per-call cost,
+    # phi of every key, and per-row cost)
     t0 = time.perf_counter()
     orc.oracle_forward(q, k, v, F, S, c["T_c"], c["T_o"], rows=np.arange(4))
     t4 = time.perf_counter() - t0
-    n = int(max(1, min(N, 4 * per_step_budget / max(t4, 1e-3))))
+    t0 = time.perf_counter()
+    orc.oracle_forward(q, k, v, F, S, c["T_c"], c["T_o"], rows=np.arange(36))
+    t36 = time.perf_counter() - t0
+    per_row = max((t36 - t4) / 32, 1e-6)
+    fixed = max(t4 - 4 * per_row, 0.0)
+    n = int(max(1, min(N, (per_step_budget - fixed) / per_row)))
     times = []
     for i in range(args.warmup + args.steps):
         rows = np.sort(rng.choice(N, n, replace=False))
