@@ -286,6 +286,18 @@ __device__ __forceinline__ float ex2(float x) {
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
+// packed fp32x2 arithmetic (sm_100): two lanes of a 64-bit register pair
+__device__ __forceinline__ uint64_t pack_f32x2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+// (x0, x1) = (a0, a1) * b + c, a0 / a1 given as raw fp32 bits
+__device__ __forceinline__ void fma_f32x2(uint32_t a0, uint32_t a1, uint64_t b, uint64_t c, float& x0, float& x1) {
+  asm("{\n\t.reg .b64 sa, sx;\n\tmov.b64 sa, {%2, %3};\n\tfma.rn.f32x2 sx, sa, %4, %5;\n\tmov.b64 {%0, %1}, sx;\n\t}"
+      : "=f"(x0), "=f"(x1)
+      : "r"(a0), "r"(a1), "l"(b), "l"(c));
+}
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);

@@ -52,12 +52,15 @@ template <uint32_t FMA_MASK, int HALF>
 __device__ __forceinline__ float exp_pack_store(uint32_t (&s)[4][32], float scale, float neg_m, uint32_t tS) {
   float rsum[4] = {0.f, 0.f, 0.f, 0.f};  // independent partial sums
   uint32_t pk[32];
+  const uint64_t sc2 = pack_f32x2(scale, scale), nm2 = pack_f32x2(neg_m, neg_m);
 #pragma unroll
   for (int a = 2 * HALF; a < 2 * HALF + 2; ++a) {
 #pragma unroll
     for (int c = 0; c < 16; ++c) {
-      const float x0 = fmaf(__uint_as_float(s[a][2 * c]), scale, neg_m);
-      const float x1 = fmaf(__uint_as_float(s[a][2 * c + 1]), scale, neg_m);
+      // x = s * scale - m for two keys in one packed fp32x2 FMA (measured
+      // 2% faster for the whole kernel than two scalar FMAs)
+      float x0, x1;
+      fma_f32x2(s[a][2 * c], s[a][2 * c + 1], sc2, nm2, x0, x1);
       const float p0 = ((FMA_MASK >> ((2 * c) & 7)) & 1u) ? exp2_fma(x0) : ex2(x0);
       const float p1 = ((FMA_MASK >> ((2 * c + 1) & 7)) & 1u) ? exp2_fma(x1) : ex2(x1);
       const uint32_t u = pack_bf16(p0, p1);
