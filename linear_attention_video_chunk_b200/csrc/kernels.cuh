@@ -5,6 +5,10 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <mutex>
+#include <set>
+#include <utility>
+
 #include "geom.cuh"
 
 namespace rehyat {
@@ -73,6 +77,29 @@ struct StateF32Params {
   float* part_S;      // [BH, n_seg, 1, 2D, D]
   float* part_z;
 };
+
+// One-time per-device setup of a kernel before its first launch: allow
+// `smem` bytes of dynamic shared memory and, when need_regs > 0, check that
+// it compiled to exactly need_regs registers a thread.  Later launches skip
+// both calls, so launches can be captured into CUDA graphs.
+inline cudaError_t prepare_kernel_once(const void* func, int smem, int need_regs) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  static std::mutex mu;
+  static std::set<std::pair<const void*, int>> done;
+  std::lock_guard<std::mutex> lock(mu);
+  if (done.count({func, dev})) return cudaSuccess;
+  if (need_regs > 0) {
+    cudaFuncAttributes fa;
+    e = cudaFuncGetAttributes(&fa, func);
+    if (e != cudaSuccess) return e;
+    if (fa.numRegs != need_regs) return cudaErrorInvalidConfiguration;
+  }
+  e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e == cudaSuccess) done.insert({func, dev});
+  return e;
+}
 
 // Shared-memory bytes each tensor-core kernel needs (dynamic).
 int attn_smem_bytes(int D);

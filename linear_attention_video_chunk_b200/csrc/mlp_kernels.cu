@@ -6,6 +6,7 @@
 #include <cstdint>
 
 #include "geom.cuh"
+#include "kernels.cuh"
 #include "mlp.cuh"
 #include "ptx.cuh"
 #include "tc_common.cuh"
@@ -314,7 +315,7 @@ __global__ void __launch_bounds__(MlpCfg<D>::THREADS, 1) phi_mlp_kernel(const __
 template <int D>
 static cudaError_t launch_mlp_t(const MlpParams& p, int n_maps, cudaStream_t s) {
   auto* k = phi_mlp_kernel<D>;
-  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, MlpCfg<D>::SMEM);
+  cudaError_t e = prepare_kernel_once(reinterpret_cast<const void*>(k), MlpCfg<D>::SMEM, 0);
   if (e != cudaSuccess) return e;
   k<<<n_maps * p.BH * p.groups, MlpCfg<D>::THREADS, MlpCfg<D>::SMEM, s>>>(p);
   return cudaGetLastError();

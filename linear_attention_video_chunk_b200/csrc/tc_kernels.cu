@@ -1005,11 +1005,8 @@ static cudaError_t launch_attn_t(const AttnParams& p, int n_units, cudaStream_t 
   auto* k = hybrid_chunk_attn_kernel<D, PARTS, PHI>;
   // The in-kernel register split assumes exactly REGS_LAUNCH registers per
   // thread at launch; with fewer, a warpgroup's increase could never be met.
-  cudaFuncAttributes fa;
-  cudaError_t e = cudaFuncGetAttributes(&fa, k);
-  if (e != cudaSuccess) return e;
-  if (static_cast<uint32_t>(fa.numRegs) != AttnCfg<D>::REGS_LAUNCH) return cudaErrorInvalidConfiguration;
-  e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, AttnCfg<D>::SMEM);
+  cudaError_t e = prepare_kernel_once(reinterpret_cast<const void*>(k), AttnCfg<D>::SMEM,
+                                      static_cast<int>(AttnCfg<D>::REGS_LAUNCH));
   if (e != cudaSuccess) return e;
   k<<<n_units, AttnCfg<D>::THREADS, AttnCfg<D>::SMEM, s>>>(p);
   return cudaGetLastError();
@@ -1029,7 +1026,7 @@ cudaError_t launch_attention_phi(int D, const AttnParams& p, int n_units, cudaSt
 template <int D, bool PRE = false>
 static cudaError_t launch_state_t(const StateParams& p, int n_ctas, cudaStream_t s) {
   auto* k = phi_state_kernel<D, PRE>;
-  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, StCfg<D>::SMEM);
+  cudaError_t e = prepare_kernel_once(reinterpret_cast<const void*>(k), StCfg<D>::SMEM, 0);
   if (e != cudaSuccess) return e;
   k<<<n_ctas, StCfg<D>::THREADS, StCfg<D>::SMEM, s>>>(p);
   return cudaGetLastError();

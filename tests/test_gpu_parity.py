@@ -462,3 +462,48 @@ def test_forward_host_buffers_equal_device_forward(layout):
     torch.cuda.synchronize()
     for o in outs:
         assert torch.equal(o, ref)
+
+
+def test_cuda_graph_capture_of_forward_and_steps():
+    """The workspace entry points allocate nothing and never synchronise, so
+    a forward and a chain of recurrent steps capture into one CUDA graph;
+    replays give the eager results bit for bit."""
+    B, H, d, F, S, Tc, To = 1, 2, 128, 6, 130, 2, 1
+    q, k, v = (x.cuda() for x in inputs.make_qkv(B, H, F * S, d, 150, rms_qk=True))
+    ws = R.alloc_workspace(R.workspace_bytes(B, H, F, S, d, Tc, To), "cuda")
+    y_eager = R.forward(q, k, v, F, S, Tc, To, workspace=ws).clone()
+    steps = []
+    for t in range(-(-F // Tc)):
+        f0, w0, cf, qf, ef = R.step_frames(t, F, Tc, To)
+        steps.append((q[:, :, f0 * S:(f0 + qf) * S].contiguous(), k[:, :, w0 * S:(f0 + qf) * S].contiguous(),
+                      v[:, :, w0 * S:(f0 + qf) * S].contiguous(), qf, cf, ef))
+    sws = R.alloc_workspace(max(R.step_workspace_bytes(B, H, S, d, s[3], s[4], s[5]) for s in steps), "cuda")
+    Sst = torch.zeros(B, H, 2 * d, d, device="cuda")
+    zst = torch.zeros(B, H, 2 * d, device="cuda")
+    outs = [torch.empty_like(s[0]) for s in steps]
+
+    def run(y):
+        R.forward(q, k, v, F, S, Tc, To, out=y, workspace=ws)
+        Sst.zero_()
+        zst.zero_()
+        for (qc, kc, vc, qf, cf, ef), o in zip(steps, outs):
+            R.step(qc, kc, vc, Sst, zst, S, qf, cf, ef, out=o, workspace=sws)
+
+    y = torch.empty_like(q)
+    run(y)  # eager pass (also loads every kernel before capture)
+    steps_eager = [o.clone() for o in outs]
+    S_eager = Sst.clone()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        run(y)
+    y.zero_()
+    for o in outs:
+        o.zero_()
+    g.replay()
+    g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(y, y_eager)
+    for o, oe in zip(outs, steps_eager):
+        assert torch.equal(o, oe)
+    assert torch.equal(Sst, S_eager)
