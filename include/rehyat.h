@@ -18,17 +18,21 @@
  *   - tokens are frame-major: j = f * S_tok + spatial index; N = F * S_tok.
  *   - the last chunk is ragged when F is not a multiple of chunk_frames.
  *   - phi(x) = [psi(x), psi(x)^2] with psi = 1 + elu on both q and k (P = 2,
- *     D' = 2d): the only concrete psi the paper gives.
+ *     D' = 2d): the only concrete psi the paper gives.  The learned maps of
+ *     §4.3 / §7.1 (two-layer MLP, separate phi_q and phi_k) are the
+ *     rehyat_phi_mlp / _phi / _mlp entry points below.
  *   - softmax weight exp(q.k / sqrt(d)).
  *   - every call computes the §3.3 (causal / recurrent) sets, so the parallel
  *     form and the step form compute the same function; rehyat_forward_ex
  *     also offers the §3.2 bidirectional sets.
  *
  * Conventions for every entry point:
- *   - Tensors are dense, row-major, in DEVICE memory owned by the caller:
- *     q, k, v, out are [B, H, N, d] (d fastest).  bf16 entry points take
- *     `const void*` pointing at IEEE bfloat16 data; _f32 ones take float.
- *     All device pointers must be 16-byte aligned (TMA requirement).
+ *   - Tensors are dense, row-major, in DEVICE memory owned by the caller
+ *     (rehyat_forward_host alone takes host q, k, v, out): q, k, v, out are
+ *     [B, H, N, d] (d fastest), or [B, N, H, d] where a `layout` argument
+ *     says so.  bf16 entry points take `const void*` pointing at IEEE
+ *     bfloat16 data; _f32 ones take float.  All device pointers must be
+ *     16-byte aligned (TMA requirement).
  *   - d must be 64 or 128 (REHYAT_EUNSUPPORTED otherwise).
  *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
  *     stream).  Calls are asynchronous: they validate, launch and return;
@@ -42,6 +46,10 @@
  *     invalid), and rehyat_device_status() reports REHYAT_ETIMEOUT.
  *   - Results are deterministic: no atomics on the data path.
  *   - Multiple calls may run concurrently on different streams.
+ *   - CUDA graphs: the entry points that take a caller workspace allocate
+ *     nothing and never synchronise the host, so their launches can be
+ *     captured into a CUDA graph.  Make one eager call per kernel variant
+ *     and device first (it sets the kernel's shared-memory limit once).
  */
 #ifndef REHYAT_H
 #define REHYAT_H
@@ -114,8 +122,8 @@ int rehyat_forward_attention(const void* q, const void* k, const void* v,
 #define REHYAT_SETS_CAUSAL 0        /* §3.3 recurrent sets: T^L_t = { j < lo_t } (rehyat_forward) */
 #define REHYAT_SETS_BIDIRECTIONAL 1 /* §3.2 sets with overlap: T^L_t = T - T^S_t (earlier and later keys) */
 
-/* Tensor layouts of rehyat_forward_ex (q, k, v and out share one). */
-#define REHYAT_LAYOUT_BHND 0  /* [B, H, N, d]: the layout of every other entry point */
+/* Tensor layouts (q, k, v and out share one). */
+#define REHYAT_LAYOUT_BHND 0  /* [B, H, N, d]: the layout of the entry points without a layout argument */
 #define REHYAT_LAYOUT_BNHD 1  /* [B, N, H, d]: heads interleaved per token, as a DiT's
                                  attention projection writes them (no transpose needed) */
 
@@ -141,7 +149,7 @@ int rehyat_forward_ex(const void* q, const void* k, const void* v,
  * P = 2).  Per head h and row x (d wide):
  *   u   = W2[h] relu(W1[h] x + b1[h]) + b2[h]     (hidden width 2d)
  *   phi = [1 + elu(u[0:d]), (1 + elu(u[d:2d]))^2]  (2d wide, non-negative)
- * The pages fix neither the hidden width nor the output non-linearity; this
+ * The paper fixes neither the hidden width nor the output non-linearity; this
  * reading keeps phi non-negative (§3.1) and gives about 2.4 M parameters per
  * block for 12 heads at d = 128 (the paper's figure).  With W1 = [I; -I],
  * W2 = [[I, -I]; [I, -I]] and zero biases it is the fixed phi.

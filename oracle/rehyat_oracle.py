@@ -73,7 +73,7 @@ def phi_mlp(x, W1, b1, W2, b2):
     """Learned feature map ("ReHyAt", §4.3 Training specification and §7.1
     Training Details): a two-layer MLP with degree-2 polynomial features,
     phi(x) = [psi_1(x)^1, psi_2(x)^2] (the §3.2 feature-map equation, P = 2).
-    The pages fix neither the hidden width nor the output non-linearity; the
+    The paper fixes neither the hidden width nor the output non-linearity; the
     reading taken here is hidden width 2d and psi_p = 1 + elu of the MLP
     outputs, which keeps phi non-negative (§3.1) and gives the paper's
     parameter count.
