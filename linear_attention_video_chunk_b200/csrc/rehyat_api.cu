@@ -16,6 +16,7 @@
 namespace rehyat {
 cudaError_t read_and_clear_device_error(unsigned int* v);
 cudaError_t read_and_clear_device_error_mlp(unsigned int* v);
+cudaError_t read_and_clear_device_error_states(unsigned int* v);
 }
 
 namespace {
@@ -947,10 +948,11 @@ REHYAT_API int rehyat_exp2_fma(const float* x, float* y, int64_t n, void* stream
 REHYAT_API int rehyat_device_status(unsigned int* detail) {
   unsigned int v = 0;
   if (cudaDeviceSynchronize() != cudaSuccess) return REHYAT_ECUDA;
-  unsigned int v_mlp = 0;
+  unsigned int v_mlp = 0, v_states = 0;
   if (read_and_clear_device_error(&v) != cudaSuccess) return REHYAT_ECUDA;
   if (read_and_clear_device_error_mlp(&v_mlp) != cudaSuccess) return REHYAT_ECUDA;
-  v |= v_mlp;
+  if (read_and_clear_device_error_states(&v_states) != cudaSuccess) return REHYAT_ECUDA;
+  v |= v_mlp | v_states;
   if (detail != nullptr) *detail = v;
   return v == 0 ? REHYAT_OK : REHYAT_ETIMEOUT;
 }
