@@ -225,12 +225,28 @@ int rehyat_forward_host(const void* q_host, const void* k_host, const void* v_ho
                         int chunk_frames, int overlap_frames, int sets, int layout,
                         void* out_host, void* workspace, size_t workspace_bytes, void* stream);
 
-/* fp32 forward (SIMT fp32 throughout, accurate exp); same sets and layout.
- * Meant for small problems and tight-tolerance checks; any size is legal. */
+/* fp32 forward (SIMT fp32 throughout, accurate exp) over the §3.3 causal
+ * sets, [B, H, N, d] float tensors.  Meant for small problems and
+ * tight-tolerance checks; any size is legal. */
 int rehyat_forward_f32(const float* q, const float* k, const float* v,
                        int B, int H, int F, int S_tok, int d,
                        int chunk_frames, int overlap_frames,
                        float* out, void* stream);
+
+/* fp32 counterparts of the learned-feature calls, for tight-tolerance checks:
+ *   rehyat_phi_mlp_f32: the feature map of rehyat_phi_mlp in fp32 (no bf16
+ *     rounding of the hidden layer or of phi); x [B, H, N, d], W1 [H, 2d, d],
+ *     b1 [H, 2d], W2 [H, 2d, 2d], b2 [H, 2d] float, phi [B, H, N, 2d] float.
+ *   rehyat_forward_phi_f32: rehyat_forward_f32 with precomputed features
+ *     phi_q, phi_k [B, H, N, 2d] float in place of the fixed phi. */
+int rehyat_phi_mlp_f32(const float* x, int B, int H, int N, int d,
+                       const float* W1, const float* b1, const float* W2, const float* b2,
+                       float* phi, void* stream);
+int rehyat_forward_phi_f32(const float* q, const float* k, const float* v,
+                           const float* phi_q, const float* phi_k,
+                           int B, int H, int F, int S_tok, int d,
+                           int chunk_frames, int overlap_frames,
+                           float* out, void* stream);
 
 /* Diagnostic form of rehyat_forward: runs the same fused tensor-core kernel
  * but writes the unnormalised terms of the §3.2 joint normaliser instead of

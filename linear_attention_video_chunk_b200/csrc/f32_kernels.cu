@@ -84,12 +84,20 @@ __global__ void __launch_bounds__(256) attn_f32_kernel(const AttnF32Params p) {
 #pragma unroll
     for (int i = 0; i < PER; ++i) aL[i] = 0.f;
     float nl = 0.f;
+    const float* fq = p.phi_q ? p.phi_q + (static_cast<size_t>(bh) * p.g.N_q + row) * (2 * D) : nullptr;
 #pragma unroll
     for (int idx = 0; idx < PER; ++idx) {
       for (int src = 0; src < 32; ++src) {
         const float x = __shfl_sync(kFull, qv[idx], src);
         const int dim = idx * 32 + src;
-        const float f1 = psi_f32(x), f2 = f1 * f1;
+        float f1, f2;
+        if (fq != nullptr) {  // precomputed (learned) features of q
+          f1 = fq[dim];
+          f2 = fq[D + dim];
+        } else {
+          f1 = psi_f32(x);
+          f2 = f1 * f1;
+        }
         nl += f1 * zp[dim] + f2 * zp[D + dim];
         const float* s1 = Sp + static_cast<size_t>(dim) * D;
         const float* s2 = Sp + static_cast<size_t>(D + dim) * D;
@@ -121,9 +129,15 @@ __global__ void __launch_bounds__(256) chunk_state_f32_kernel(const StateF32Para
   const float* vb = p.v + static_cast<size_t>(bh) * p.sg.N_k * D;
   const int dim = e < D ? e : e - D;
   float acc = 0.f;
+  const float* fk = p.phi_k ? p.phi_k + static_cast<size_t>(bh) * p.sg.N_k * 2 * D : nullptr;
   for (int j = a; j < b; ++j) {
-    float f = psi_f32(kb[static_cast<size_t>(j) * D + dim]);
-    if (e >= D) f = f * f;
+    float f;
+    if (fk != nullptr) {  // precomputed (learned) features of k
+      f = fk[static_cast<size_t>(j) * 2 * D + e];
+    } else {
+      f = psi_f32(kb[static_cast<size_t>(j) * D + dim]);
+      if (e >= D) f = f * f;
+    }
     acc += (c == D) ? f : f * vb[static_cast<size_t>(j) * D + c];
   }
   const size_t po = static_cast<size_t>(bh) * p.sg.n_seg + s;  // nsplit == 1
@@ -154,7 +168,57 @@ __global__ void phi_kernel(const void* x, int x_f32, void* y, int y_f32, long lo
   }
 }
 
+// Learned feature map (two-layer MLP, degree-2 features), fp32: a block
+// takes MLP_ROWS rows; the hidden layer relu(W1 x + b1) goes through shared
+// memory, then phi = [psi(u_1), psi(u_2)^2] of u = W2 h + b2.
+constexpr int MLP_ROWS = 4;
+__global__ void __launch_bounds__(256) phi_mlp_f32_kernel(const float* __restrict__ x, long long rows, int N, int H,
+                                                          int d, const float* __restrict__ W1,
+                                                          const float* __restrict__ b1,
+                                                          const float* __restrict__ W2,
+                                                          const float* __restrict__ b2, float* __restrict__ phi) {
+  extern __shared__ float hid[];  // [MLP_ROWS][2d]
+  const int d2 = 2 * d;
+  const long long r0 = static_cast<long long>(blockIdx.x) * MLP_ROWS;
+  for (int i = threadIdx.x; i < MLP_ROWS * d2; i += blockDim.x) {
+    const int rr = i / d2, j = i % d2;
+    const long long row = r0 + rr;
+    float h = 0.f;
+    if (row < rows) {
+      const int head = static_cast<int>((row / N) % H);
+      const float* w = W1 + (static_cast<size_t>(head) * d2 + j) * d;
+      const float* xr = x + row * d;
+      float a = b1[static_cast<size_t>(head) * d2 + j];
+      for (int c = 0; c < d; ++c) a = fmaf(w[c], xr[c], a);
+      h = fmaxf(a, 0.f);
+    }
+    hid[rr * d2 + j] = h;
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < MLP_ROWS * d2; i += blockDim.x) {
+    const int rr = i / d2, o = i % d2;
+    const long long row = r0 + rr;
+    if (row >= rows) continue;
+    const int head = static_cast<int>((row / N) % H);
+    const float* w = W2 + (static_cast<size_t>(head) * d2 + o) * d2;
+    float u = b2[static_cast<size_t>(head) * d2 + o];
+    for (int j = 0; j < d2; ++j) u = fmaf(w[j], hid[rr * d2 + j], u);
+    const float f = psi_f32(u);
+    phi[row * d2 + o] = (o < d) ? f : f * f;
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_phi_mlp_f32(const float* x, long long rows, int N, int H, int d, const float* W1,
+                               const float* b1, const float* W2, const float* b2, float* phi, cudaStream_t s) {
+  const long long blocks = (rows + MLP_ROWS - 1) / MLP_ROWS;
+  if (blocks <= 0) return cudaSuccess;
+  if (blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
+  phi_mlp_f32_kernel<<<static_cast<unsigned>(blocks), 256, MLP_ROWS * 2 * d * sizeof(float), s>>>(
+      x, rows, N, H, d, W1, b1, W2, b2, phi);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_attention_f32(const AttnF32Params& p, int n_chunks, cudaStream_t s) {
   const int row_blocks = cdiv(p.g.step ? p.g.N_q : p.g.chunk_tok, 8);

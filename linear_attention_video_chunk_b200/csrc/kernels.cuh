@@ -67,6 +67,7 @@ struct AttnF32Params {
   const float* z;     // z_t at z[bh*z_bh + t*z_t]
   long long z_bh, z_t;
   float* out;         // [BH, N_q, D]
+  const float* phi_q; // optional [BH, N_q, 2D] precomputed phi(q) (null: the fixed phi of q)
 };
 
 struct StateF32Params {
@@ -76,6 +77,7 @@ struct StateF32Params {
   const float* v;
   float* part_S;      // [BH, n_seg, 1, 2D, D]
   float* part_z;
+  const float* phi_k; // optional [BH, N_k, 2D] precomputed phi(k) (null: the fixed phi of k)
 };
 
 // One-time per-device setup of a kernel before its first launch: allow
@@ -134,5 +136,9 @@ cudaError_t launch_attention_f32(const AttnF32Params& p, int n_chunks, cudaStrea
 cudaError_t launch_chunk_state_f32(const StateF32Params& p, cudaStream_t s);
 cudaError_t launch_phi(const void* x, int x_f32, void* y, int y_f32, long long rows, int d,
                        cudaStream_t s);
+// Learned feature map in fp32 SIMT: x [BH, N, d] (head = (row / N) % H),
+// W1 [H, 2d, d], b1 [H, 2d], W2 [H, 2d, 2d], b2 [H, 2d] -> phi [BH, N, 2d].
+cudaError_t launch_phi_mlp_f32(const float* x, long long rows, int N, int H, int d, const float* W1,
+                               const float* b1, const float* W2, const float* b2, float* phi, cudaStream_t s);
 
 }  // namespace rehyat

@@ -723,8 +723,39 @@ REHYAT_API int rehyat_chunk_states(const void* k, const void* v, int B, int H, i
   return run_states(k, v, P, static_cast<uint8_t*>(ws.p), S, z, s);
 }
 
+namespace {
+// fp32 forward with optional precomputed features (null: the fixed phi).
+int run_forward_f32(const float* q, const float* k, const float* v, const float* phi_q, const float* phi_k, int B,
+                    int H, int F, int S_tok, int d, int chunk_frames, int overlap_frames, float* out, void* stream);
+}  // namespace
+
 REHYAT_API int rehyat_forward_f32(const float* q, const float* k, const float* v, int B, int H, int F, int S_tok,
                                   int d, int chunk_frames, int overlap_frames, float* out, void* stream) {
+  return run_forward_f32(q, k, v, nullptr, nullptr, B, H, F, S_tok, d, chunk_frames, overlap_frames, out, stream);
+}
+
+REHYAT_API int rehyat_forward_phi_f32(const float* q, const float* k, const float* v, const float* phi_q,
+                                      const float* phi_k, int B, int H, int F, int S_tok, int d, int chunk_frames,
+                                      int overlap_frames, float* out, void* stream) {
+  if (check_ptr(phi_q) || check_ptr(phi_k)) return REHYAT_EINVAL;
+  return run_forward_f32(q, k, v, phi_q, phi_k, B, H, F, S_tok, d, chunk_frames, overlap_frames, out, stream);
+}
+
+REHYAT_API int rehyat_phi_mlp_f32(const float* x, int B, int H, int N, int d, const float* W1, const float* b1,
+                                  const float* W2, const float* b2, float* phi, void* stream) {
+  if (B < 1 || H < 1 || N < 1) return REHYAT_EINVAL;
+  int st = check_d(d);
+  if (st != REHYAT_OK) return st;
+  if (check_ptr(x) || check_ptr(W1) || check_ptr(b1) || check_ptr(W2) || check_ptr(b2) || check_ptr(phi))
+    return REHYAT_EINVAL;
+  const long long rows = static_cast<long long>(B) * H * N;
+  if (rows * d > (1LL << 46)) return REHYAT_EINVAL;
+  return cuda_status(launch_phi_mlp_f32(x, rows, N, H, d, W1, b1, W2, b2, phi, static_cast<cudaStream_t>(stream)));
+}
+
+namespace {
+int run_forward_f32(const float* q, const float* k, const float* v, const float* phi_q, const float* phi_k, int B,
+                    int H, int F, int S_tok, int d, int chunk_frames, int overlap_frames, float* out, void* stream) {
   FwdPlan P;
   int st = plan_forward(B, H, F, S_tok, d, chunk_frames, overlap_frames, &P);
   if (st != REHYAT_OK) return st;
@@ -739,7 +770,7 @@ REHYAT_API int rehyat_forward_f32(const float* q, const float* k, const float* v
   float* pz = reinterpret_cast<float*>(w + P.f32_off_pz);
   float* Sf = reinterpret_cast<float*>(w + P.f32_off_S);
   float* zt = reinterpret_cast<float*>(w + P.f32_off_zt);
-  StateF32Params sp;
+  StateF32Params sp{};
   sp.sg = SegGeom{P.N, P.chunk_tok, P.ovl_tok, P.n_seg, 1, 0, 0};
   sp.BH = P.BH;
   sp.D = P.D;
@@ -747,11 +778,12 @@ REHYAT_API int rehyat_forward_f32(const float* q, const float* k, const float* v
   sp.v = v;
   sp.part_S = pS;
   sp.part_z = pz;
+  sp.phi_k = phi_k;
   st = cuda_status(launch_chunk_state_f32(sp, s));
   if (st != REHYAT_OK) return st;
   st = cuda_status(launch_state_scan(pS, pz, P.BH, P.n_seg, 1, P.nc, P.D, nullptr, nullptr, Sf, zt, s));
   if (st != REHYAT_OK) return st;
-  AttnF32Params ap;
+  AttnF32Params ap{};
   ap.g = ChunkGeom{P.N, P.N, P.chunk_tok, P.ovl_tok, P.nc, 0};
   ap.BH = P.BH;
   ap.D = P.D;
@@ -763,8 +795,10 @@ REHYAT_API int rehyat_forward_f32(const float* q, const float* k, const float* v
   ap.z_bh = 2LL * P.D * P.nc;
   ap.z_t = 2LL * P.D;
   ap.out = out;
+  ap.phi_q = phi_q;
   return cuda_status(launch_attention_f32(ap, P.nc, s));
 }
+}  // namespace
 
 // ---------------------------------------------------------------------------
 // recurrent form
@@ -896,7 +930,7 @@ REHYAT_API int rehyat_step_f32(const float* q_c, const float* k_c, const float* 
   if (st != REHYAT_OK) return st;
   if (check_qkvo(q_c, k_c, v_c, out_c) || check_ptr(state_S) || check_ptr(state_z)) return REHYAT_EINVAL;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  AttnF32Params ap;
+  AttnF32Params ap{};
   ap.g = ChunkGeom{P.Nq, P.Nk, P.Nq, 0, 1, 1};
   ap.BH = P.BH;
   ap.D = P.D;
@@ -914,7 +948,7 @@ REHYAT_API int rehyat_step_f32(const float* q_c, const float* k_c, const float* 
   st = ws.alloc(P.f32_bytes);
   if (st != REHYAT_OK) return st;
   uint8_t* w = static_cast<uint8_t*>(ws.p);
-  StateF32Params sp;
+  StateF32Params sp{};
   sp.sg = SegGeom{P.Nk, 0, 0, 1, 1, 1, P.evict_tok};
   sp.BH = P.BH;
   sp.D = P.D;

@@ -46,6 +46,8 @@ _SIGS = {
     "rehyat_step_phi": [_vp] * 8 + [_I] * 7 + [_vp, _c_size, _vp],
     "rehyat_forward_host_workspace_bytes": [_I, _I, _I, _I, _I, _I, _I, _I, ctypes.POINTER(_c_size)],
     "rehyat_forward_host": [_vp, _vp, _vp] + [_I] * 9 + [_vp, _vp, _c_size, _vp],
+    "rehyat_phi_mlp_f32": [_vp, _I, _I, _I, _I, _vp, _vp, _vp, _vp, _vp, _vp],
+    "rehyat_forward_phi_f32": [_vp] * 5 + [_I] * 7 + [_vp, _vp],
 }
 _RESTYPES = {"rehyat_status_string": ctypes.c_char_p}
 
@@ -401,6 +403,33 @@ def step_phi(q_c, k_c, v_c, phi_q_c, phi_k_c, state_S, state_z, S_tok, q_frames,
     _check(lib().rehyat_step_phi(_p(q_c), _p(k_c), _p(v_c), _p(phi_q_c), _p(phi_k_c), _p(state_S), _p(state_z),
                                  _p(out), B, H, S_tok, d, q_frames, ctx_frames, evict_frames, _p(ws),
                                  ws.numel() if ws is not None else 0, _stream()), "rehyat_step_phi")
+    return out
+
+
+def phi_mlp_f32(x, W1, b1, W2, b2, out=None):
+    """rehyat_phi_mlp_f32: the learned feature map in fp32, x [B,H,N,d]
+    float, weights float -> phi [B,H,N,2d] float."""
+    _need(x, torch.float32, "x")
+    B, H, N, d = x.shape
+    for n, t, shape in (("W1", W1, (H, 2 * d, d)), ("b1", b1, (H, 2 * d)), ("W2", W2, (H, 2 * d, 2 * d)),
+                        ("b2", b2, (H, 2 * d))):
+        _need(t, torch.float32, n, len(shape))
+        if tuple(t.shape) != shape:
+            raise ValueError(f"{n} must be {shape}")
+    out = torch.empty((B, H, N, 2 * d), dtype=torch.float32, device=x.device) if out is None else out
+    _check(lib().rehyat_phi_mlp_f32(_p(x), B, H, N, d, _p(W1), _p(b1), _p(W2), _p(b2), _p(out), _stream()),
+           "rehyat_phi_mlp_f32")
+    return out
+
+
+def forward_phi_f32(q, k, v, phi_q, phi_k, F, S_tok, chunk_frames, overlap_frames, out=None):
+    """rehyat_forward_phi_f32: the fp32 forward with precomputed features."""
+    for n, t in (("q", q), ("k", k), ("v", v), ("phi_q", phi_q), ("phi_k", phi_k)):
+        _need(t, torch.float32, n)
+    B, H, N, d = _shape(q, F, S_tok)
+    out = torch.empty_like(q) if out is None else out
+    _check(lib().rehyat_forward_phi_f32(_p(q), _p(k), _p(v), _p(phi_q), _p(phi_k), B, H, F, S_tok, d, chunk_frames,
+                                        overlap_frames, _p(out), _stream()), "rehyat_forward_phi_f32")
     return out
 
 

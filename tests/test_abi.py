@@ -196,3 +196,11 @@ def test_forward_host_validation(lib):
     ex = ctypes.c_size_t(0)
     lib.rehyat_forward_ex_workspace_bytes(1, 12, 21, 1560, 128, 3, 1, 0, ctypes.byref(ex))
     assert R.forward_host_workspace_bytes(1, 12, 21, 1560, 128, 3, 1) == ex.value + 4 * 12 * 32760 * 128 * 2
+
+
+def test_f32_learned_phi_validation(lib):
+    assert lib.rehyat_phi_mlp_f32(0, 1, 1, 8, 64, 16, 16, 16, 16, 16, None) == R.EINVAL
+    assert lib.rehyat_phi_mlp_f32(16, 1, 1, 8, 96, 16, 16, 16, 16, 16, None) == R.EUNSUPPORTED
+    assert lib.rehyat_phi_mlp_f32(16, 1, 1, 0, 64, 16, 16, 16, 16, 16, None) == R.EINVAL
+    assert lib.rehyat_forward_phi_f32(16, 16, 16, 0, 16, 1, 1, 4, 8, 64, 2, 1, 16, None) == R.EINVAL
+    assert lib.rehyat_forward_phi_f32(16, 16, 16, 16, 24, 1, 1, 4, 8, 64, 2, 1, 16, None) == R.EINVAL

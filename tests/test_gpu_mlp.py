@@ -228,3 +228,36 @@ def test_step_phi_streamed_matches_oracle(F, S, Tc, To):
     assert_bf16_close(y, ref, "step_phi vs oracle")
     yf = np64(R.forward_phi(qd, kd, vd, Pqd, Pkd, F, S, Tc, To))
     assert np.linalg.norm(y - yf) / np.linalg.norm(yf) <= 5e-3
+
+
+F32_TOL = 1e-5
+
+
+@pytest.mark.parametrize("B,H,N,d,kind,seed", [(1, 2, 300, 128, "random", 60), (2, 1, 70, 64, "near_identity", 61)])
+def test_phi_mlp_f32_matches_oracle(B, H, N, d, kind, seed):
+    """The fp32 feature map against the oracle's fp64 MLP, relative L2 <= 1e-5."""
+    x = inputs.make_qkv(B, H, N, d, seed, dtype="f32", scale=0.5)[0]
+    w = tuple(t.float() for t in inputs.make_mlp_weights(H, d, seed, "q", kind))
+    y = R.phi_mlp_f32(x.cuda(), *(t.cuda() for t in w)).cpu().double().numpy()
+    ref = _oracle_phi(x, w)
+    err = np.sqrt(((y - ref) ** 2).sum()) / np.sqrt((ref ** 2).sum())
+    assert err <= F32_TOL, err
+
+
+@pytest.mark.parametrize("F,S,Tc,To", [(4, 64, 2, 1), (5, 40, 2, 3), (6, 30, 3, 0)])
+def test_forward_phi_f32_matches_oracle(F, S, Tc, To):
+    """The fp32 learned-feature forward (fp32 feature map, then the fp32
+    hybrid attention with those features) against the oracle end to end,
+    relative L2 <= 1e-5 per (b, h)."""
+    B, H, d = 1, 2, 64
+    q, k, v = inputs.make_qkv(B, H, F * S, d, 62, dtype="f32", scale=0.5)
+    wq = tuple(t.float() for t in inputs.make_mlp_weights(H, d, 62, "q", "random"))
+    wk = tuple(t.float() for t in inputs.make_mlp_weights(H, d, 62, "k", "random"))
+    qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+    Pq = R.phi_mlp_f32(qd, *(t.cuda() for t in wq))
+    Pk = R.phi_mlp_f32(kd, *(t.cuda() for t in wk))
+    y = R.forward_phi_f32(qd, kd, vd, Pq, Pk, F, S, Tc, To).cpu().double().numpy()
+    ref = orc.oracle_forward(q, k, v, F, S, Tc, To, phi_q=_oracle_phi(q, wq), phi_k=_oracle_phi(k, wk))
+    num = np.sqrt(((y - ref) ** 2).sum(axis=(-2, -1)))
+    den = np.sqrt((ref ** 2).sum(axis=(-2, -1)))
+    assert (num / den).max() <= F32_TOL, (num / den).max()
