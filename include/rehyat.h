@@ -190,6 +190,16 @@ int rehyat_forward_mlp(const void* q, const void* k, const void* v,
                        int chunk_frames, int overlap_frames, int sets, int layout,
                        void* out, void* workspace, size_t workspace_bytes, void* stream);
 
+/* rehyat_step with a tensor layout (REHYAT_LAYOUT_BHND or _BNHD: q_c, k_c,
+ * v_c and out_c share it; the state is always [B, H, 2d, d] / [B, H, 2d])
+ * and an optional caller workspace (NULL: stream-ordered scratch, else
+ * rehyat_step_workspace_bytes(...) bytes, 256-byte aligned). */
+int rehyat_step_ex(const void* q_c, const void* k_c, const void* v_c,
+                   float* state_S, float* state_z, void* out_c,
+                   int B, int H, int S_tok, int d,
+                   int q_frames, int ctx_frames, int evict_frames, int layout,
+                   void* workspace, size_t workspace_bytes, void* stream);
+
 /* rehyat_step with precomputed feature maps (e.g. rehyat_phi_mlp of the
  * chunk's q and of its window's k): phi_q_c [B, H, Lq, 2d] bf16 replaces the
  * fixed phi of q_c in the linear term, phi_k_c [B, H, Lk, 2d] bf16 that of

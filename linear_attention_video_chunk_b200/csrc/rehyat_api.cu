@@ -819,7 +819,8 @@ namespace {
 // state.  phi_q / phi_k (optional): precomputed features of the chunk's
 // queries and of the window's keys ([B, H, Lq, 2d], [B, H, Lk, 2d]).
 int run_step(const void* q_c, const void* k_c, const void* v_c, const void* phi_q, const void* phi_k, float* state_S,
-             float* state_z, void* out_c, const StepPlan& P, uint8_t* w, cudaStream_t s) {
+             float* state_z, void* out_c, const StepPlan& P, uint8_t* w, cudaStream_t s,
+             int layout = REHYAT_LAYOUT_BHND) {
   __nv_bfloat16* hi = reinterpret_cast<__nv_bfloat16*>(w + P.off_hi);
   __nv_bfloat16* lo = reinterpret_cast<__nv_bfloat16*>(w + P.off_lo);
   int st = cuda_status(launch_state_split(state_S, static_cast<long long>(P.BH) * 2 * P.D * P.D, hi, lo, s));
@@ -827,17 +828,21 @@ int run_step(const void* q_c, const void* k_c, const void* v_c, const void* phi_
   AttnParams ap;
   std::memset(&ap, 0, sizeof(ap));
   const long long d_ = P.D, H_ = P.H, Nq_ = P.Nq, Nk_ = P.Nk, D2 = 2LL * P.D;
-  if (!make_map4(&ap.tm_q, q_c, P.D, P.Nq, P.H, P.B, d_, Nq_ * d_, H_ * Nq_ * d_, 128) ||
-      !make_map4(&ap.tm_k, k_c, P.D, P.Nk, P.H, P.B, d_, Nk_ * d_, H_ * Nk_ * d_, 128) ||
-      !make_map4(&ap.tm_v, v_c, P.D, P.Nk, P.H, P.B, d_, Nk_ * d_, H_ * Nk_ * d_, 128) ||
+  // element strides of a row, a head and a batch for q / out (rows Nq) and k / v (rows Nk)
+  const bool bnhd = layout == REHYAT_LAYOUT_BNHD;
+  const long long q_rs = bnhd ? H_ * d_ : d_, q_hs = bnhd ? d_ : Nq_ * d_, q_bs = H_ * Nq_ * d_;
+  const long long k_rs = bnhd ? H_ * d_ : d_, k_hs = bnhd ? d_ : Nk_ * d_, k_bs = H_ * Nk_ * d_;
+  if (!make_map4(&ap.tm_q, q_c, P.D, P.Nq, P.H, P.B, q_rs, q_hs, q_bs, 128) ||
+      !make_map4(&ap.tm_k, k_c, P.D, P.Nk, P.H, P.B, k_rs, k_hs, k_bs, 128) ||
+      !make_map4(&ap.tm_v, v_c, P.D, P.Nk, P.H, P.B, k_rs, k_hs, k_bs, 128) ||
       !make_map(&ap.tm_hi, hi, P.D, 2LL * P.D, P.BH, 128) || !make_map(&ap.tm_lo, lo, P.D, 2LL * P.D, P.BH, 128))
     return REHYAT_ECUDA;
   ap.g = ChunkGeom{P.Nq, P.Nk, P.Nq, 0, 1, 1};
   ap.BH = P.BH;
   ap.H = P.H;
-  ap.o_sb = H_ * Nq_ * d_;
-  ap.o_sh = Nq_ * d_;
-  ap.o_sr = d_;
+  ap.o_sb = q_bs;
+  ap.o_sh = q_hs;
+  ap.o_sr = q_rs;
   ap.pairs = P.pairs;
   ap.state_mul = 1;
   ap.scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(P.D));
@@ -854,9 +859,9 @@ int run_step(const void* q_c, const void* k_c, const void* v_c, const void* phi_
   if (st != REHYAT_OK || P.evict_tok == 0) return st;
   StateParams sp;
   std::memset(&sp, 0, sizeof(sp));
-  if ((phi_k == nullptr && !make_map4(&sp.tm_k, k_c, P.D, P.Nk, P.H, P.B, d_, Nk_ * d_, H_ * Nk_ * d_, 64)) ||
+  if ((phi_k == nullptr && !make_map4(&sp.tm_k, k_c, P.D, P.Nk, P.H, P.B, k_rs, k_hs, k_bs, 64)) ||
       (phi_k != nullptr && !make_map4(&sp.tm_phik, phi_k, D2, P.Nk, P.H, P.B, D2, Nk_ * D2, H_ * Nk_ * D2, 64)) ||
-      !make_map4(&sp.tm_v, v_c, P.D, P.Nk, P.H, P.B, d_, Nk_ * d_, H_ * Nk_ * d_, 64))
+      !make_map4(&sp.tm_v, v_c, P.D, P.Nk, P.H, P.B, k_rs, k_hs, k_bs, 64))
     return REHYAT_ECUDA;
   sp.sg = SegGeom{P.Nk, 0, 0, 1, P.nsplit, 1, P.evict_tok};
   sp.BH = P.BH;
@@ -905,6 +910,28 @@ REHYAT_API int rehyat_step_phi(const void* q_c, const void* k_c, const void* v_c
     if (workspace_bytes < P.bytes) return REHYAT_ENOMEM;
   }
   return run_step(q_c, k_c, v_c, phi_q_c, phi_k_c, state_S, state_z, out_c, P, static_cast<uint8_t*>(workspace), s);
+}
+
+REHYAT_API int rehyat_step_ex(const void* q_c, const void* k_c, const void* v_c, float* state_S, float* state_z,
+                              void* out_c, int B, int H, int S_tok, int d, int q_frames, int ctx_frames,
+                              int evict_frames, int layout, void* workspace, size_t workspace_bytes, void* stream) {
+  StepPlan P;
+  int st = plan_step(B, H, S_tok, d, q_frames, ctx_frames, evict_frames, &P);
+  if (st != REHYAT_OK) return st;
+  if (layout != REHYAT_LAYOUT_BHND && layout != REHYAT_LAYOUT_BNHD) return REHYAT_EINVAL;
+  if (check_qkvo(q_c, k_c, v_c, out_c) || check_ptr(state_S) || check_ptr(state_z)) return REHYAT_EINVAL;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  WsGuard own(s);
+  if (workspace == nullptr) {
+    st = own.alloc(P.bytes);
+    if (st != REHYAT_OK) return st;
+    workspace = own.p;
+  } else {
+    if (reinterpret_cast<uintptr_t>(workspace) % 256 != 0) return REHYAT_EINVAL;
+    if (workspace_bytes < P.bytes) return REHYAT_ENOMEM;
+  }
+  return run_step(q_c, k_c, v_c, nullptr, nullptr, state_S, state_z, out_c, P, static_cast<uint8_t*>(workspace), s,
+                  layout);
 }
 
 REHYAT_API int rehyat_step(const void* q_c, const void* k_c, const void* v_c, float* state_S, float* state_z,

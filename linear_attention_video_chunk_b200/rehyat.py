@@ -47,6 +47,7 @@ _SIGS = {
     "rehyat_forward_host_workspace_bytes": [_I, _I, _I, _I, _I, _I, _I, _I, ctypes.POINTER(_c_size)],
     "rehyat_forward_host": [_vp, _vp, _vp] + [_I] * 9 + [_vp, _vp, _c_size, _vp],
     "rehyat_phi_mlp_f32": [_vp, _I, _I, _I, _I, _vp, _vp, _vp, _vp, _vp, _vp],
+    "rehyat_step_ex": [_vp] * 6 + [_I] * 8 + [_vp, _c_size, _vp],
     "rehyat_forward_phi_f32": [_vp] * 5 + [_I] * 7 + [_vp, _vp],
 }
 _RESTYPES = {"rehyat_status_string": ctypes.c_char_p}
@@ -382,6 +383,30 @@ def step(q_c, k_c, v_c, state_S, state_z, S_tok, q_frames, ctx_frames, evict_fra
     ws = alloc_workspace(nb, q_c.device) if workspace is None else workspace
     _check(lib().rehyat_step_ws(_p(q_c), _p(k_c), _p(v_c), _p(state_S), _p(state_z), _p(out), B, H, S_tok, d,
                                 q_frames, ctx_frames, evict_frames, _p(ws), ws.numel(), _stream()), "rehyat_step_ws")
+    return out
+
+
+def step_ex(q_c, k_c, v_c, state_S, state_z, S_tok, q_frames, ctx_frames, evict_frames, layout="bhnd", out=None,
+            workspace=None):
+    """rehyat_step_ex: one chunk of the recurrent form on [B,H,L,d] ("bhnd")
+    or [B,L,H,d] ("bnhd") tensors."""
+    for n, t in (("q_c", q_c), ("k_c", k_c), ("v_c", v_c)):
+        _need(t, torch.bfloat16, n)
+    _need(state_S, torch.float32, "state_S")
+    _need(state_z, torch.float32, "state_z", 3)
+    if layout == "bhnd":
+        B, H, Lq, d = q_c.shape
+        Lk = k_c.shape[2]
+    else:
+        B, Lq, H, d = q_c.shape
+        Lk = k_c.shape[1]
+    if Lq != q_frames * S_tok or Lk != (ctx_frames + q_frames) * S_tok:
+        raise ValueError("q_c / k_c lengths do not match the frame counts")
+    out = torch.empty_like(q_c) if out is None else out
+    ws = workspace
+    _check(lib().rehyat_step_ex(_p(q_c), _p(k_c), _p(v_c), _p(state_S), _p(state_z), _p(out), B, H, S_tok, d,
+                                q_frames, ctx_frames, evict_frames, LAYOUTS[layout], _p(ws),
+                                ws.numel() if ws is not None else 0, _stream()), "rehyat_step_ex")
     return out
 
 

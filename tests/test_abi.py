@@ -204,3 +204,12 @@ def test_f32_learned_phi_validation(lib):
     assert lib.rehyat_phi_mlp_f32(16, 1, 1, 0, 64, 16, 16, 16, 16, 16, None) == R.EINVAL
     assert lib.rehyat_forward_phi_f32(16, 16, 16, 0, 16, 1, 1, 4, 8, 64, 2, 1, 16, None) == R.EINVAL
     assert lib.rehyat_forward_phi_f32(16, 16, 16, 16, 24, 1, 1, 4, 8, 64, 2, 1, 16, None) == R.EINVAL
+
+
+def test_step_ex_validation(lib):
+    def se(layout=0, ws=0, nb=0, q=16):
+        return lib.rehyat_step_ex(q, 16, 16, 16, 16, 16, 1, 1, 8, 64, 2, 1, 1, layout, ws, nb, None)
+    assert se(layout=2) == R.EINVAL
+    assert se(q=0) == R.EINVAL
+    assert se(ws=256, nb=1) == R.ENOMEM
+    assert se(ws=272, nb=1 << 30) == R.EINVAL

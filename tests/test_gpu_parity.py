@@ -507,3 +507,24 @@ def test_cuda_graph_capture_of_forward_and_steps():
     for o, oe in zip(outs, steps_eager):
         assert torch.equal(o, oe)
     assert torch.equal(Sst, S_eager)
+
+
+
+def test_step_bnhd_layout_equals_bhnd_bitwise():
+    """rehyat_step_ex on [B, L, H, d] chunks returns the [B, H, L, d] step's
+    output transposed, bit for bit, and carries the same state."""
+    B, H, d, F, S, Tc, To = 1, 3, 128, 7, 64, 2, 1
+    q, k, v = (x.cuda() for x in inputs.make_qkv(B, H, F * S, d, 160, rms_qk=True))
+    t = lambda x: x.transpose(1, 2).contiguous()
+    S1 = torch.zeros(B, H, 2 * d, d, device="cuda")
+    z1 = torch.zeros(B, H, 2 * d, device="cuda")
+    S2, z2 = S1.clone(), z1.clone()
+    for c in range(-(-F // Tc)):
+        f0, w0, cf, qf, ef = R.step_frames(c, F, Tc, To)
+        qc = q[:, :, f0 * S:(f0 + qf) * S].contiguous()
+        kc = k[:, :, w0 * S:(f0 + qf) * S].contiguous()
+        vc = v[:, :, w0 * S:(f0 + qf) * S].contiguous()
+        y1 = R.step(qc, kc, vc, S1, z1, S, qf, cf, ef)
+        y2 = R.step_ex(t(qc), t(kc), t(vc), S2, z2, S, qf, cf, ef, layout="bnhd")
+        assert torch.equal(t(y2), y1)
+    assert torch.equal(S1, S2) and torch.equal(z1, z2)
