@@ -93,8 +93,9 @@ struct AttnCfg {
   static constexpr int B_FULL = 1;
   static constexpr int B_EMPTY = B_FULL + NSLOTS;
   static constexpr int B_S = B_EMPTY + NSLOTS;   // [2] scores ready in TMEM
-  static constexpr int B_P = B_S + 2;            // [2] P written to TMEM
-  static constexpr int B_O = B_P + 2;            // [2] last P.V done
+  static constexpr int B_P = B_S + 2;            // [2] first 64 keys of P written to TMEM
+  static constexpr int B_P1 = B_P + 2;           // [2] last 64 keys of P written to TMEM
+  static constexpr int B_O = B_P1 + 2;           // [2] last P.V done
   static constexpr int B_PHI = B_O + 2;          // [2] scaled phi(Q) written to TMEM
   static constexpr int B_LIN = B_PHI + 2;        // [2] linear MMA done
   static constexpr int B_FIN = B_LIN + 2;        // MMA drain
@@ -118,7 +119,7 @@ struct AttnCfg {
 };
 
 // events: softmax of tile X (lane 0 of warp 4X): 0+5X S ready seen, 1+5X S in
-// registers, 2+5X max done, 3+5X P stored, 4+5X P released; MMA issuer:
+// registers, 2+5X max done, 3+5X first P half released, 4+5X P released; MMA issuer:
 // 10+X P_X seen, 12+X S_X(j+1) issued, 14 unit start (j = 0), Q and K_0 in
 // (j = 1), K_{j+1} in (j + 2), 15 P_A.V_j issued
 
@@ -170,6 +171,7 @@ __global__ void __launch_bounds__(384, 1) hybrid_chunk_attn_kernel(const __grid_
     for (int x = 0; x < 2; ++x) {
       mbar_init(BAR(C::B_S + x), 1);
       mbar_init(BAR(C::B_P + x), 4);           // one arrive per softmax warp
+      mbar_init(BAR(C::B_P1 + x), 4);
       mbar_init(BAR(C::B_O + x), 1);
       mbar_init(BAR(C::B_PHI + x), 4);
       mbar_init(BAR(C::B_LIN + x), 1);
@@ -270,15 +272,17 @@ __global__ void __launch_bounds__(384, 1) hybrid_chunk_attn_kernel(const __grid_
         const float alpha = need ? ex2(m_used - mnew) : 1.f;
         m_used = mnew;
         const float neg_m = -m_used;
+        // P is released in two 64-key halves, so the first half's P.V runs
+        // on the tensor core while the second half's exponentials are taken.
         // Full tiles may send a share of the exponentials to the FMA pipe;
         // the window's partial last tile stays on ex2 (masked keys give 0).
         float rs = (valid >= 128) ? exp_pack_store<REHYAT_EXP2_FMA_MASK, 0>(s, p.scale_log2, neg_m, tS)
                                   : exp_pack_store<0u, 0>(s, p.scale_log2, neg_m, tS);
-        rs += (valid >= 128) ? exp_pack_store<REHYAT_EXP2_FMA_MASK, 1>(s, p.scale_log2, neg_m, tS)
-                             : exp_pack_store<0u, 1>(s, p.scale_log2, neg_m, tS);
         if (warp_need && j > 0) {
           // O holds tiles 0..j-1 (their P.V completed before S_j was
           // signalled) and must move to the new shift before P_j.V_j.
+          // (Done after the first half's exponentials, whose scores no
+          // longer occupy registers.)
 #pragma unroll
           for (int a = 0; a < D / 32; ++a) {
             uint32_t ov[32];
@@ -289,10 +293,12 @@ __global__ void __launch_bounds__(384, 1) hybrid_chunk_attn_kernel(const __grid_
             for (int c = 0; c < 32; ++c) ov[c] = __float_as_uint(__uint_as_float(ov[c]) * alpha);
             tmem_st32(tO + 32 * a, ov);
           }
-          tmem_st_wait();
         }
-        if (wl == 0 && lane == 0) TRACE(3 + 5 * X, j);
         warp_release(BAR(C::B_P + X), lane);
+        if (wl == 0 && lane == 0) TRACE(3 + 5 * X, j);
+        rs += (valid >= 128) ? exp_pack_store<REHYAT_EXP2_FMA_MASK, 1>(s, p.scale_log2, neg_m, tS)
+                             : exp_pack_store<0u, 1>(s, p.scale_log2, neg_m, tS);
+        warp_release(BAR(C::B_P1 + X), lane);
         if (wl == 0 && lane == 0) TRACE(4 + 5 * X, j);
         l = l * alpha + rs;
       }
@@ -512,12 +518,15 @@ __global__ void __launch_bounds__(384, 1) hybrid_chunk_attn_kernel(const __grid_
                  (first && kk == 0) ? 0u : 1u);
         }
       };
-      // O_X += P_X V_j once the softmax warps have released P_X
+      // O_X += P_X V_j, each 64-key half once the softmax warps have
+      // released it
       auto issue_PV = [&](int X, uint32_t vb, int j) -> bool {
         if (!mbar_wait(BAR(C::B_P + X), j & 1, abort)) return false;
         TRACE(10 + X, j);
         tc_fence_after();
         issue_PV_half(tmem + 256 + X * D, tmem + X * 128, vb, j == 0, 0);
+        if (!mbar_wait(BAR(C::B_P1 + X), j & 1, abort)) return false;
+        tc_fence_after();
         issue_PV_half(tmem + 256 + X * D, tmem + X * 128, vb, j == 0, 1);
         return true;
       };
