@@ -213,3 +213,37 @@ def test_step_ex_validation(lib):
     assert se(q=0) == R.EINVAL
     assert se(ws=256, nb=1) == R.ENOMEM
     assert se(ws=272, nb=1 << 30) == R.EINVAL
+
+
+def _header_signatures():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    src = re.sub(r"//[^\n]*", "", src)
+    out = {}
+    for ret, name, args in re.findall(r"\b([\w ]+?\*?)\s*\b(rehyat_\w+)\s*\(([^)]*)\)\s*;", src):
+        a = args.strip()
+        out[name] = (ret.strip(), [] if a in ("", "void") else [x.strip() for x in a.split(",")])
+    return out
+
+
+def _ctype_of(decl):
+    """Coarse ctypes class of one C parameter declaration."""
+    if "*" in decl:
+        return "ptr"
+    t = decl.rsplit(" ", 1)[0].strip()
+    return {"int": "int", "int64_t": "int64", "size_t": "size_t", "float": "float"}[t]
+
+
+def test_binding_argtypes_match_the_header():
+    """Every binding's ctypes argument list has the header's arity and, per
+    position, the same kind (pointer / int / int64 / size_t), so no call marshals
+    an argument into the wrong slot."""
+    kind = {ctypes.c_void_p: "ptr", ctypes.c_int: "int", ctypes.c_int64: "int64", ctypes.c_size_t: "size_t",
+            ctypes.c_float: "float"}
+    sigs = _header_signatures()
+    assert len(sigs) == len(declared_functions())
+    for name, (ret, params) in sigs.items():
+        want = [_ctype_of(p) for p in params]
+        got = [kind.get(t, "ptr") for t in R._SIGS[name]]
+        assert got == want, (name, got, want)
+        assert (R._RESTYPES.get(name, ctypes.c_int) is ctypes.c_char_p) == ret.startswith("const char")
