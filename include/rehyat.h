@@ -190,10 +190,20 @@ int rehyat_forward_mlp(const void* q, const void* k, const void* v,
                        int chunk_frames, int overlap_frames, int sets, int layout,
                        void* out, void* workspace, size_t workspace_bytes, void* stream);
 
-/* rehyat_step with a tensor layout (REHYAT_LAYOUT_BHND or _BNHD: q_c, k_c,
- * v_c and out_c share it; the state is always [B, H, 2d, d] / [B, H, 2d])
- * and an optional caller workspace (NULL: stream-ordered scratch, else
- * rehyat_step_workspace_bytes(...) bytes, 256-byte aligned). */
+/* rehyat_step (one chunk of the §3.3 recurrent form) with a tensor layout
+ * and an optional caller workspace.
+ *   layout  REHYAT_LAYOUT_BHND: q_c / out_c [B, H, Lq, d], k_c / v_c
+ *           [B, H, Lk, d]; REHYAT_LAYOUT_BNHD: [B, Lq, H, d] / [B, Lk, H, d]
+ *           (Lq = q_frames * S_tok, Lk = (ctx_frames + q_frames) * S_tok);
+ *           all bf16 device, caller-owned, 16-byte aligned.  The state is
+ *           always [B, H, 2d, d] / [B, H, 2d] fp32, updated in place.
+ *   workspace  NULL: stream-ordered scratch allocated and freed on `stream`;
+ *           else rehyat_step_workspace_bytes(...) bytes, 256-byte aligned.
+ * Frame bookkeeping, results and asynchrony as rehyat_step: the output is
+ * the [B, H, Lq, d] step's output in the chosen layout, bit for bit.
+ * Returns REHYAT_EINVAL for an unknown layout, null / misaligned pointers or
+ * bad sizes, REHYAT_ENOMEM for a workspace smaller than required; nothing is
+ * launched after a validation failure. */
 int rehyat_step_ex(const void* q_c, const void* k_c, const void* v_c,
                    float* state_S, float* state_z, void* out_c,
                    int B, int H, int S_tok, int d,
