@@ -647,25 +647,49 @@ def run_sweep(args):
 # reference arm: the fp64 oracle on the host cores                             #
 # --------------------------------------------------------------------------- #
 def run_reference(args):
+    """The fp64 oracle, as it stands, on the host cores: the same workload
+    (config, heads override, set mode, feature map) as our arm, each step a
+    random query-row sample (all heads) sized so the whole run lasts about
+    --ref-budget seconds."""
     rank, world, _ = dist_env()
     if rank != 0:
         return
     from linear_attention_video_chunk_b200 import inputs
-    c = dict(CONFIGS["wan13b"])
+    c = dict(CONFIGS[args.config])
+    if args.heads:
+        c["H"] = args.heads
+        c["workload"] += f" (H overridden to {args.heads})"
     B, H, d, F, S = (c[k] for k in ("B", "H", "d", "F", "S_tok"))
     q, k, v = inputs.make_qkv(B, H, F * S, d, c["seed"], rms_qk=True)
     import numpy as np
     import oracle.rehyat_oracle as orc
+    feats = {}
+    if args.phi == "mlp":
+        # the learned map's features of every token, from the same seeded weights
+        for which, x in (("q", q), ("k", k)):
+            W1, b1, W2, b2 = (t.float().numpy() for t in inputs.make_mlp_weights(H, d, c["seed"], which))
+            xs = x.float().numpy()
+            feats["phi_" + which] = np.stack([np.stack([orc.phi_mlp(xs[b, h], W1[h], b1[h], W2[h], b2[h])
+                                                        for h in range(H)]) for b in range(B)])
+        c["workload"] += " (learned phi: 2-layer MLP, degree-2 features)"
+    if args.sets != "causal":
+        c["workload"] += f" ({args.sets} sets)"
+    if args.layout != "bhnd":
+        c["workload"] += " ([B, N, H, d] layout)"
+
+    def call(rows):
+        orc.oracle_forward(q, k, v, F, S, c["T_c"], c["T_o"], mode=args.sets, rows=rows, **feats)
+
     N = F * S
     rng = np.random.default_rng(11)
-    per_step_budget = max(0.2, 150.0 / max(1, args.steps + args.warmup))
+    per_step_budget = max(0.05, args.ref_budget / max(1, args.steps + args.warmup))
     # size each step's row sample from two calibration calls (per-call cost,
     # phi of every key, and per-row cost)
     t0 = time.perf_counter()
-    orc.oracle_forward(q, k, v, F, S, c["T_c"], c["T_o"], rows=np.arange(4))
+    call(np.arange(4))
     t4 = time.perf_counter() - t0
     t0 = time.perf_counter()
-    orc.oracle_forward(q, k, v, F, S, c["T_c"], c["T_o"], rows=np.arange(36))
+    call(np.arange(36))
     t36 = time.perf_counter() - t0
     per_row = max((t36 - t4) / 32, 1e-6)
     fixed = max(t4 - 4 * per_row, 0.0)
@@ -674,11 +698,11 @@ def run_reference(args):
     for i in range(args.warmup + args.steps):
         rows = np.sort(rng.choice(N, n, replace=False))
         t0 = time.perf_counter()
-        orc.oracle_forward(q, k, v, F, S, c["T_c"], c["T_o"], rows=rows)
+        call(rows)
         if i >= args.warmup:
             times.append(time.perf_counter() - t0)
     sec = sum(times) / len(times)
-    val = n / sec
+    val = B * n / sec
     line = {
         "impl": "reference", "metric": METRIC, "value": val, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": sec * 1e3, "higher_is_better": True, "scaling": "weak",
@@ -709,6 +733,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end leg (profiling runs)")
     ap.add_argument("--heads", type=int, default=0, help="override H (smaller profiling cases)")
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work for cpu_baseline")
+    ap.add_argument("--ref-budget", type=float, default=150.0,
+                    help="seconds of oracle work for the whole --impl reference run")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -39,3 +39,43 @@ def test_wan13b_work_figures():
     assert w["attn_flops"] == 12 * (4 * 128 * pairs + 2 * 256 * 129 * n_lin)
     # q, k, v, out once (bf16) + per chunk the bf16 hi and lo states and fp32 z
     assert w["attn_bytes"] == 12 * 32760 * 128 * 2 * 4 + 12 * 7 * 256 * (128 * 4 + 4)
+
+
+# --------------------------------------------------------------------------- #
+# the reference arm (the oracle on the host cores) keeps the line contract     #
+# --------------------------------------------------------------------------- #
+import json
+import os
+import subprocess
+import sys
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _bench(*args, env=None):
+    e = dict(os.environ)
+    e.update(env or {})
+    return subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), *args], capture_output=True, text=True,
+                          timeout=300, cwd=ROOT, env=e)
+
+
+def test_reference_arm_prints_one_contract_line():
+    r = _bench("--impl", "reference", "--steps", "1", "--warmup", "3", "--heads", "1", "--ref-budget", "1")
+    assert r.returncode == 0, r.stderr
+    lines = [l for l in r.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    j = json.loads(lines[0])
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+                "scaling", "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"):
+        assert key in j, key
+    assert j["impl"] == "reference" and j["value"] > 0 and j["steps"] == 1
+    assert j["cpu_baseline"]["kind"] == "oracle" and j["cpu_baseline"]["value"] == j["value"]
+    assert j["e2e"] == {"value": j["value"], "unit": j["unit"], "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+    assert j["config"]["H"] == 1 and "workload" in j["config"]
+
+
+def test_reference_arm_other_ranks_exit_quietly():
+    r = _bench("--impl", "reference", "--steps", "1", "--warmup", "3", "--heads", "1", "--ref-budget", "1",
+               env={"RANK": "1", "WORLD_SIZE": "2", "LOCAL_RANK": "1"})
+    assert r.returncode == 0, r.stderr
+    assert not [l for l in r.stdout.splitlines() if l.startswith("{")]
