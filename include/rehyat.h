@@ -373,6 +373,15 @@ int rehyat_phi(const void* x, int x_dtype, void* y, int y_dtype,
  * treated as -125).  x, y: n floats in device memory. */
 int rehyat_exp2_fma(const float* x, float* y, int64_t n, void* stream);
 
+/* Diagnostic for the failure path: launches one warp that waits on a
+ * barrier nothing ever completes.  The wait is bounded like every device
+ * wait in this library (2 s of GPU time); it then records the timeout in the
+ * device error word and the kernel returns, so rehyat_device_status()
+ * reports REHYAT_ETIMEOUT once and later calls run normally.  gave_up: NULL
+ * or one device int, set to 1 when the wait gave up (0 had it completed).
+ * Returns REHYAT_ECUDA if the launch fails. */
+int rehyat_wait_probe(int* gave_up, void* stream);
+
 /* Synchronises the current device and reports whether any kernel of this
  * library recorded a device-side error since the last call (REHYAT_ETIMEOUT
  * when a bounded wait ran out), then clears the record.  *detail (optional)

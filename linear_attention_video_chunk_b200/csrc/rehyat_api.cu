@@ -17,6 +17,7 @@ namespace rehyat {
 cudaError_t read_and_clear_device_error(unsigned int* v);
 cudaError_t read_and_clear_device_error_mlp(unsigned int* v);
 cudaError_t read_and_clear_device_error_states(unsigned int* v);
+cudaError_t launch_wait_probe(int* gave_up, cudaStream_t s);
 }
 
 namespace {
@@ -1004,6 +1005,10 @@ REHYAT_API int rehyat_phi(const void* x, int x_dtype, void* y, int y_dtype, int6
 REHYAT_API int rehyat_exp2_fma(const float* x, float* y, int64_t n, void* stream) {
   if (x == nullptr || y == nullptr || n < 1) return REHYAT_EINVAL;
   return cuda_status(launch_exp2_fma(x, y, n, static_cast<cudaStream_t>(stream)));
+}
+
+REHYAT_API int rehyat_wait_probe(int* gave_up, void* stream) {
+  return cuda_status(launch_wait_probe(gave_up, static_cast<cudaStream_t>(stream)));
 }
 
 REHYAT_API int rehyat_device_status(unsigned int* detail) {

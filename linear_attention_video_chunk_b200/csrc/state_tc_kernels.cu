@@ -277,7 +277,29 @@ __global__ void __launch_bounds__(StCfg<D>::THREADS, 1) phi_state_kernel(const _
   }
 }
 
+// Failure-path check: one warp waits on an mbarrier that nothing ever
+// arrives on.  The bounded wait gives up after its limit, records the timeout
+// in this unit's device error word and returns, so the host reads
+// REHYAT_ETIMEOUT and the context stays usable.
+__global__ void wait_probe_kernel(int* gave_up) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_word;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar), 1);
+    abort_word = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  const bool ok = mbar_wait(smem_u32(&bar), 0, &abort_word);
+  if (threadIdx.x == 0 && gave_up != nullptr) *gave_up = ok ? 0 : 1;
+}
+
 }  // namespace
+
+cudaError_t launch_wait_probe(int* gave_up, cudaStream_t s) {
+  wait_probe_kernel<<<1, 32, 0, s>>>(gave_up);
+  return cudaGetLastError();
+}
 
 int state_smem_bytes(int D) { return D == 128 ? StCfg<128>::SMEM : StCfg<64>::SMEM; }
 

@@ -48,6 +48,7 @@ _SIGS = {
     "rehyat_forward_host": [_vp, _vp, _vp] + [_I] * 9 + [_vp, _vp, _c_size, _vp],
     "rehyat_phi_mlp_f32": [_vp, _I, _I, _I, _I, _vp, _vp, _vp, _vp, _vp, _vp],
     "rehyat_step_ex": [_vp] * 6 + [_I] * 8 + [_vp, _c_size, _vp],
+    "rehyat_wait_probe": [_vp, _vp],
     "rehyat_forward_phi_f32": [_vp] * 5 + [_I] * 7 + [_vp, _vp],
 }
 _RESTYPES = {"rehyat_status_string": ctypes.c_char_p}
@@ -502,6 +503,15 @@ def exp2_fma(x: torch.Tensor) -> torch.Tensor:
     y = torch.empty_like(x)
     _check(lib().rehyat_exp2_fma(_p(x), _p(y), x.numel(), _stream()), "rehyat_exp2_fma")
     return y
+
+
+def wait_probe(gave_up=None):
+    """rehyat_wait_probe: one warp waits on a barrier nothing completes; the
+    bounded wait gives up after its limit.  gave_up: optional int32 device
+    tensor of one element, set to 1 when the wait gave up."""
+    if gave_up is not None:
+        _need(gave_up, torch.int32, "gave_up", 1)
+    _check(lib().rehyat_wait_probe(_p(gave_up), _stream()), "rehyat_wait_probe")
 
 
 def device_status() -> int:

@@ -528,3 +528,53 @@ def test_step_bnhd_layout_equals_bhnd_bitwise():
         y2 = R.step_ex(t(qc), t(kc), t(vc), S2, z2, S, qf, cf, ef, layout="bnhd")
         assert torch.equal(t(y2), y1)
     assert torch.equal(S1, S2) and torch.equal(z1, z2)
+
+
+def test_bounded_wait_gives_up_and_context_survives():
+    """Failure detection without a fault: a device wait on a barrier that
+    nothing completes gives up after its limit (2 s), the host reads
+    REHYAT_ETIMEOUT once, and the next forward runs and matches the oracle."""
+    import time
+    assert R.device_status() == R.OK
+    flag = torch.zeros(1, dtype=torch.int32, device="cuda")
+    t0 = time.perf_counter()
+    R.wait_probe(flag)
+    torch.cuda.synchronize()
+    dt = time.perf_counter() - t0
+    assert flag.item() == 1
+    assert 1.5 < dt < 60, dt
+    assert R.device_status() == R.ETIMEOUT
+    assert R.device_status() == R.OK  # read and cleared
+    B, H, d, F, S, Tc, To = 1, 1, 128, 4, 64, 2, 1
+    q, k, v = inputs.make_qkv(B, H, F * S, d, 170, rms_qk=True)
+    y = R.forward(q.cuda(), k.cuda(), v.cuda(), F, S, Tc, To)
+    assert_bf16_close(np64(y), orc.oracle_forward(q, k, v, F, S, Tc, To), "after the timeout")
+    assert R.device_status() == R.OK
+
+
+def test_step_state_checkpoint_through_host_resumes_bitwise():
+    """The recurrent state (S, z) is the checkpoint: copied to the host after
+    chunk t and back into fresh device buffers, the video continues with
+    bit-identical outputs and final state."""
+    B, H, d, F, S, Tc, To = 1, 2, 128, 9, 64, 2, 1
+    q, k, v = (x.cuda() for x in inputs.make_qkv(B, H, F * S, d, 171, rms_qk=True))
+    nc = -(-F // Tc)
+
+    def run(stop=None):
+        Sst = torch.zeros(B, H, 2 * d, d, device="cuda")
+        zst = torch.zeros(B, H, 2 * d, device="cuda")
+        outs = []
+        for t in range(nc):
+            if t == stop:
+                Sh, zh = Sst.cpu(), zst.cpu()
+                del Sst, zst
+                Sst, zst = Sh.cuda(), zh.cuda()
+            f0, w0, cf, qf, ef = R.step_frames(t, F, Tc, To)
+            outs.append(R.step(q[:, :, f0 * S:(f0 + qf) * S].contiguous(), k[:, :, w0 * S:(f0 + qf) * S].contiguous(),
+                               v[:, :, w0 * S:(f0 + qf) * S].contiguous(), Sst, zst, S, qf, cf, ef))
+        return torch.cat(outs, dim=2), Sst, zst
+
+    y0, S0, z0 = run()
+    for stop in (1, 3, nc - 1):
+        y1, S1, z1 = run(stop)
+        assert torch.equal(y0, y1) and torch.equal(S0, S1) and torch.equal(z0, z1), stop
