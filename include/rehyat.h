@@ -338,6 +338,10 @@ int rehyat_step(const void* q_c, const void* k_c, const void* v_c,
                 int B, int H, int S_tok, int d,
                 int q_frames, int ctx_frames, int evict_frames, void* stream);
 
+/* Device scratch bytes one rehyat_step call of this shape needs (partial
+ * states of the evicted keys and the state's bf16 hi/lo split); written to
+ * *bytes.  Validates the arguments as rehyat_step does (REHYAT_EINVAL,
+ * REHYAT_EUNSUPPORTED); launches nothing. */
 int rehyat_step_workspace_bytes(int B, int H, int S_tok, int d,
                                 int q_frames, int ctx_frames, int evict_frames,
                                 size_t* bytes);

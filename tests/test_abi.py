@@ -247,3 +247,33 @@ def test_binding_argtypes_match_the_header():
         got = [kind.get(t, "ptr") for t in R._SIGS[name]]
         assert got == want, (name, got, want)
         assert (R._RESTYPES.get(name, ctypes.c_int) is ctypes.c_char_p) == ret.startswith("const char")
+
+
+def _undocumented(lines):
+    """Declarations with no comment block closing right above them or above
+    the contiguous group of declaration / #define lines they belong to."""
+    out = []
+    for i, l in enumerate(lines):
+        m = re.match(r"^\s*(?:const\s+)?\w[\w\s*]*?\b(rehyat_\w+)\s*\(", l)
+        if not m or l.lstrip().startswith(("*", "/*")):
+            continue
+        j = i - 1
+        while j >= 0 and lines[j].strip() and not lines[j].strip().endswith("*/"):
+            j -= 1
+        if j < 0 or not lines[j].strip().endswith("*/"):
+            out.append(m.group(1))
+    return out
+
+
+def test_every_declaration_is_documented():
+    """Each entry point in the header has a comment block right above it, or
+    belongs to a group of declarations (or a #define) that the block right
+    above the group documents."""
+    lines = open(HEADER).read().splitlines()
+    assert not _undocumented(lines), _undocumented(lines)
+    # the check itself catches a declaration whose comment is removed
+    k = next(i for i, l in enumerate(lines) if l.startswith("int rehyat_step_ex("))
+    j = k - 1
+    while not lines[j].lstrip().startswith("/*"):
+        j -= 1
+    assert "rehyat_step_ex" in _undocumented(lines[:j] + [""] + lines[k:])
