@@ -489,6 +489,8 @@ REHYAT_API int rehyat_forward_attention(const void* q, const void* k, const void
 REHYAT_API int rehyat_forward_ws(const void* q, const void* k, const void* v, int B, int H, int F, int S_tok,
                                  int d, int chunk_frames, int overlap_frames, void* out, void* workspace,
                                  size_t workspace_bytes, void* stream) {
+  // every pointer is checked before the first stage launches anything
+  if (check_qkvo(q, k, v, out)) return REHYAT_EINVAL;
   int st = rehyat_forward_states(k, v, B, H, F, S_tok, d, chunk_frames, overlap_frames, workspace,
                                  workspace_bytes, stream);
   if (st != REHYAT_OK) return st;

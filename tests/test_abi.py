@@ -277,3 +277,40 @@ def test_every_declaration_is_documented():
     while not lines[j].lstrip().startswith("/*"):
         j -= 1
     assert "rehyat_step_ex" in _undocumented(lines[:j] + [""] + lines[k:])
+
+
+# Pointer arguments that may be NULL by contract (besides `stream`): the
+# workspace of the calls that then allocate stream-ordered scratch.
+_NULLABLE = {(n, "workspace") for n in ("rehyat_forward_ex", "rehyat_forward_phi", "rehyat_forward_mlp",
+                                         "rehyat_step_ex", "rehyat_step_phi")}
+_SIZES = dict(B=1, H=1, F=4, S_tok=8, N=32, d=64, chunk_frames=2, overlap_frames=1, sets=0, layout=0, q_frames=2,
+              ctx_frames=1, evict_frames=1, x_dtype=0, y_dtype=0, rows=4, n=4, workspace_bytes=1 << 30)
+
+
+@pytest.mark.skipif(__import__("torch").cuda.is_available(),
+                    reason="passes fake device addresses; host-only check")
+def test_each_required_pointer_is_validated(lib):
+    """For every entry point and every required pointer argument: with valid
+    sizes, that pointer NULL and every other pointer a fake aligned address,
+    the call returns REHYAT_EINVAL before any CUDA call (a call that went on
+    would fail in CUDA here, with no device, and return something else)."""
+    out_bytes = ctypes.create_string_buffer(64)
+    missing = []
+    for name, (ret, params) in _header_signatures().items():
+        if name in ("rehyat_wait_probe", "rehyat_device_status", "rehyat_status_string"):
+            continue
+        names = [p.replace("*", " ").split()[-1] for p in params]
+        for k, p in enumerate(params):
+            if "*" not in p or names[k] == "stream" or (name, names[k]) in _NULLABLE:
+                continue
+            vals = []
+            for i, (q, pn) in enumerate(zip(params, names)):
+                if "*" not in q:
+                    vals.append(_SIZES[pn])
+                elif i == k or pn == "stream":
+                    vals.append(None)
+                else:
+                    vals.append(ctypes.addressof(out_bytes) if pn == "bytes" else 0x10000)
+            if getattr(lib, name)(*vals) != R.EINVAL:
+                missing.append((name, names[k]))
+    assert not missing, missing
