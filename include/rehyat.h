@@ -367,14 +367,18 @@ int rehyat_step_f32(const float* q_c, const float* k_c, const float* v_c,
 #define REHYAT_DTYPE_F32 1
 
 /* §3.2 feature map phi(x) = [psi(x), psi(x)^2], psi = 1 + elu (§3.1),
- * row-wise: x [rows, d] -> y [rows, 2d].  dtype codes REHYAT_DTYPE_*. */
+ * row-wise: x [rows, d] -> y [rows, 2d], any d >= 1.  dtype codes
+ * REHYAT_DTYPE_*; x, y device memory aligned to their element size.
+ * Returns REHYAT_EINVAL for null / misaligned pointers, an unknown dtype or
+ * bad sizes. */
 int rehyat_phi(const void* x, int x_dtype, void* y, int y_dtype,
                int64_t rows, int d, void* stream);
 
 /* Diagnostic: y[i] = 2^x[i] by the FMA-pipe exponential the fused kernel uses
  * for part of its softmax weights (round-to-nearest range reduction and a
  * fitted cubic; max relative error 7.5e-5 for x in [-125, 8]; x < -125 is
- * treated as -125).  x, y: n floats in device memory. */
+ * treated as -125).  x, y: n floats in device memory (4-byte aligned);
+ * REHYAT_EINVAL for null / misaligned pointers or n < 1. */
 int rehyat_exp2_fma(const float* x, float* y, int64_t n, void* stream);
 
 /* Diagnostic for the failure path: launches one warp that waits on a

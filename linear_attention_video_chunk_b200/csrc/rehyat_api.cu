@@ -1000,12 +1000,17 @@ REHYAT_API int rehyat_phi(const void* x, int x_dtype, void* y, int y_dtype, int6
       (y_dtype != REHYAT_DTYPE_BF16 && y_dtype != REHYAT_DTYPE_F32))
     return REHYAT_EINVAL;
   if (rows > (1LL << 40) / d) return REHYAT_EINVAL;
+  // element accesses: each pointer aligned to its element size
+  if (reinterpret_cast<uintptr_t>(x) % (x_dtype == REHYAT_DTYPE_F32 ? 4 : 2) != 0 ||
+      reinterpret_cast<uintptr_t>(y) % (y_dtype == REHYAT_DTYPE_F32 ? 4 : 2) != 0)
+    return REHYAT_EINVAL;
   return cuda_status(launch_phi(x, x_dtype == REHYAT_DTYPE_F32, y, y_dtype == REHYAT_DTYPE_F32, rows, d,
                                 static_cast<cudaStream_t>(stream)));
 }
 
 REHYAT_API int rehyat_exp2_fma(const float* x, float* y, int64_t n, void* stream) {
   if (x == nullptr || y == nullptr || n < 1) return REHYAT_EINVAL;
+  if (reinterpret_cast<uintptr_t>(x) % 4 != 0 || reinterpret_cast<uintptr_t>(y) % 4 != 0) return REHYAT_EINVAL;
   return cuda_status(launch_exp2_fma(x, y, n, static_cast<cudaStream_t>(stream)));
 }
 

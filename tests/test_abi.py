@@ -294,7 +294,7 @@ def test_each_required_pointer_is_validated(lib):
     sizes, that pointer NULL and every other pointer a fake aligned address,
     the call returns REHYAT_EINVAL before any CUDA call (a call that went on
     would fail in CUDA here, with no device, and return something else)."""
-    out_bytes = ctypes.create_string_buffer(64)
+    size_out = ctypes.c_size_t(0)
     missing = []
     for name, (ret, params) in _header_signatures().items():
         if name in ("rehyat_wait_probe", "rehyat_device_status", "rehyat_status_string"):
@@ -310,7 +310,51 @@ def test_each_required_pointer_is_validated(lib):
                 elif i == k or pn == "stream":
                     vals.append(None)
                 else:
-                    vals.append(ctypes.addressof(out_bytes) if pn == "bytes" else 0x10000)
+                    vals.append(ctypes.byref(size_out) if pn == "bytes" else 0x10000)
             if getattr(lib, name)(*vals) != R.EINVAL:
                 missing.append((name, names[k]))
+    assert not missing, missing
+
+
+def test_elementwise_calls_check_element_alignment(lib):
+    assert lib.rehyat_phi(0x10001, 0, 0x10000, 0, 4, 64, None) == R.EINVAL       # bf16 x at an odd address
+    assert lib.rehyat_phi(0x10000, 1, 0x10002, 1, 4, 64, None) == R.EINVAL       # fp32 y at 2 mod 4
+    assert lib.rehyat_phi(0x10000, 2, 0x10000, 0, 4, 64, None) == R.EINVAL       # unknown dtype
+    assert lib.rehyat_exp2_fma(0x10002, 0x10000, 4, None) == R.EINVAL
+    assert lib.rehyat_exp2_fma(0x10000, 0x10000, 0, None) == R.EINVAL
+
+
+_BAD_SIZES = dict(B=[0, -1], H=[0], F=[0], S_tok=[0], N=[0], d=[96, 0], chunk_frames=[0], overlap_frames=[-1],
+                  sets=[2, -1], layout=[2, -1], q_frames=[0], ctx_frames=[-1], evict_frames=[-1, 4], x_dtype=[2],
+                  y_dtype=[2], rows=[0], n=[0])
+
+
+@pytest.mark.skipif(__import__("torch").cuda.is_available(),
+                    reason="passes fake device addresses; host-only check")
+def test_each_size_argument_is_validated(lib):
+    """For every entry point and every size / mode argument: one invalid value
+    (zero or negative counts, d outside {64, 128}, unknown set mode, layout
+    or dtype, more evicted frames than the window holds), every other argument
+    valid, returns REHYAT_EINVAL or REHYAT_EUNSUPPORTED before any CUDA call."""
+    missing = []
+    for name, (ret, params) in _header_signatures().items():
+        if name in ("rehyat_wait_probe", "rehyat_device_status", "rehyat_status_string"):
+            continue
+        names = [p.replace("*", " ").split()[-1] for p in params]
+        for k, pn in enumerate(names):
+            if "*" in params[k] or pn == "workspace_bytes":
+                continue
+            for bad in _BAD_SIZES[pn]:
+                if name == "rehyat_phi" and pn == "d" and bad > 0:
+                    continue  # the element-wise map takes any d >= 1
+                vals = []
+                for i, (q, n2) in enumerate(zip(params, names)):
+                    if "*" not in q:
+                        vals.append(bad if i == k else _SIZES[n2])
+                    elif n2 == "stream":
+                        vals.append(None)
+                    else:
+                        vals.append(ctypes.byref(ctypes.c_size_t(0)) if n2 == "bytes" else 0x10000)
+                if getattr(lib, name)(*vals) not in (R.EINVAL, R.EUNSUPPORTED):
+                    missing.append((name, pn, bad))
     assert not missing, missing
