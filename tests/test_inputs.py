@@ -32,3 +32,25 @@ def test_bf16_is_round_to_nearest_even():
     lsb = (f >> 16) & 1
     want = ((f + 0x7FFF + lsb) >> 16).astype(np.uint16)
     np.testing.assert_array_equal(got, want)
+
+
+def test_mlp_weights_shapes_streams_and_kinds():
+    """Learned-map stand-in weights: shapes and storage types the library
+    takes, one stream per (seed, map, head), near-identity = the weights
+    that make the MLP the fixed map plus small noise, random = no identity."""
+    import oracle.rehyat_oracle as orc
+    H, d = 3, 64
+    W1, b1, W2, b2 = inputs.make_mlp_weights(H, d, 5, "q")
+    assert (W1.shape, W2.shape, b1.shape, b2.shape) == ((H, 2 * d, d), (H, 2 * d, 2 * d), (H, 2 * d), (H, 2 * d))
+    assert (W1.dtype, W2.dtype, b1.dtype, b2.dtype) == (torch.bfloat16, torch.bfloat16, torch.float32, torch.float32)
+    again = inputs.make_mlp_weights(H, d, 5, "q")
+    assert all(torch.equal(a, b) for a, b in zip((W1, b1, W2, b2), again))
+    Wk = inputs.make_mlp_weights(H, d, 5, "k")[0]
+    assert not torch.equal(W1, Wk) and not torch.equal(W1[0], W1[1])
+    I1, _, I2, _ = orc.mlp_identity_weights(d)
+    dev1 = (W1.double().numpy() - I1).std()
+    dev2 = (W2.double().numpy() - I2).std()
+    assert 0.05 / d ** 0.5 < dev1 < 0.2 / d ** 0.5 and 0.05 / (2 * d) ** 0.5 < dev2 < 0.2 / (2 * d) ** 0.5
+    assert float(b1.abs().max()) < 0.1 and float(b2.abs().max()) < 0.1
+    R1 = inputs.make_mlp_weights(H, d, 5, "q", kind="random")[0].double().numpy()
+    assert abs(R1.std() - 1 / d ** 0.5) < 0.1 / d ** 0.5 and abs((R1 - I1).mean()) < 0.05
