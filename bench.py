@@ -770,6 +770,10 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    if args.gpus != world:
+        ap.error(f"--gpus {args.gpus} with {world} process(es): run N > 1 as "
+                 f"python -m torch.distributed.run --nproc-per-node N bench.py --gpus N")
     if args.impl == "reference":
         run_reference(args)
     elif args.sweep:

@@ -75,7 +75,12 @@ def test_reference_arm_prints_one_contract_line():
 
 
 def test_reference_arm_other_ranks_exit_quietly():
-    r = _bench("--impl", "reference", "--steps", "1", "--warmup", "3", "--heads", "1", "--ref-budget", "1",
-               env={"RANK": "1", "WORLD_SIZE": "2", "LOCAL_RANK": "1"})
+    r = _bench("--impl", "reference", "--gpus", "2", "--steps", "1", "--warmup", "3", "--heads", "1",
+               "--ref-budget", "1", env={"RANK": "1", "WORLD_SIZE": "2", "LOCAL_RANK": "1"})
     assert r.returncode == 0, r.stderr
     assert not [l for l in r.stdout.splitlines() if l.startswith("{")]
+
+
+def test_gpu_count_must_match_the_process_count():
+    r = _bench("--impl", "reference", "--gpus", "2", "--steps", "1", "--warmup", "3", env={"WORLD_SIZE": "1"})
+    assert r.returncode != 0 and "torch.distributed.run" in r.stderr
