@@ -75,6 +75,17 @@ def work(c, sets="causal"):
                 state_bytes=state_bytes, tokens=B * N, mlp_flops=mlp_flops, mlp_bytes=mlp_bytes)
 
 
+def recurrent_bytes(c):
+    """HBM bytes of the recurrent form over one video: every step reads its
+    chunk's queries and its whole key/value window (overlap frames again) and
+    writes its output (bf16), and reads and writes the fp32 state (S, z)."""
+    B, H, d, F, S, Tc, To = (c[k] for k in ("B", "H", "d", "F", "S_tok", "T_c", "T_o"))
+    BH, D2 = B * H, 2 * d
+    rows = sum(2 * (q1 - q0) + 2 * (hi - lo) for q0, q1, lo, hi in chunks(F, S, Tc, To))
+    n_steps = -(-F // min(Tc, F))
+    return BH * rows * d * 2 + n_steps * BH * 2 * D2 * (d + 1) * 4
+
+
 KERNEL_SOURCES = ("tc_kernels.cu", "tc_common.cuh", "ptx.cuh", "kernels.cuh", "geom.cuh")
 TRAFFIC_PROFILE = os.path.join(ROOT, "profiles", "hybrid_chunk_attn_h6_full.md")
 
@@ -195,6 +206,15 @@ def oracle_sample_rate(c, q, k, v, budget_s):
     orc.oracle_forward(q, k, v, *args, rows=rows)
     dt = time.perf_counter() - t0
     return n / dt, n, dt
+
+
+def config_dict(c, world):
+    """The workload description both arms print (identical for one workload)."""
+    tokens = c["B"] * c["F"] * c["S_tok"]
+    return {"workload": c["workload"], "B": c["B"], "H": c["H"], "d": c["d"], "F": c["F"], "S_tok": c["S_tok"],
+            "chunk_frames": c["T_c"], "overlap_frames": c["T_o"], "tokens_per_step_per_gpu": tokens,
+            "parallelism": f"replicas x{world} (no collective)",
+            "l2": "inputs larger than L2: q+k+v = %.0f MB per GPU" % (3 * tokens * c["H"] * c["d"] * 2 / 1e6)}
 
 
 # --------------------------------------------------------------------------- #
@@ -408,10 +428,7 @@ def run_ours(args):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": res["ms_step"], "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic: seeded N(0,1) Q/K/V, per-vector RMS-normalised Q/K, bf16 (no latents or weights)",
-        "config": {"workload": c["workload"], "B": c["B"], "H": c["H"], "d": c["d"], "F": c["F"],
-                   "S_tok": c["S_tok"], "chunk_frames": c["T_c"], "overlap_frames": c["T_o"],
-                   "tokens_per_step_per_gpu": w["tokens"], "parallelism": f"replicas x{world} (no collective)",
-                   "l2": "inputs larger than L2: q+k+v = %.0f MB per GPU" % (3 * w["tokens"] * c["H"] * c["d"] * 2 / 1e6)},
+        "config": config_dict(c, world),
     }
     if args.config != "recurrent" and args.sets == "causal" and args.layout == "bhnd" and args.phi == "fixed":
         achieved = w["attn_flops"] / (res["attn_ms"] / 1e3) / 1e12
@@ -429,8 +446,23 @@ def run_ours(args):
     if res.get("e2e_kind"):
         line["e2e"]["how"] = res["e2e_kind"]
     if res.get("eager_ms"):
-        line["config"]["timed_as"] = "one CUDA graph per video (27 steps x 4 kernels at 81 frames)"
-        line["config"]["eager_ms_per_video"] = res["eager_ms"]
+        line["timing"] = {"timed_as": "one CUDA graph per video (%d steps x 4 kernels)" % (-(-c["F"] // c["T_c"])),
+                          "eager_ms_per_video": res["eager_ms"]}
+    if args.config == "recurrent":
+        # a streamed video does exactly the parallel form's algorithmic work
+        # (same pairs, same linear terms, the same keys folded into the state)
+        flops = w["attn_flops"] + w["state_flops"]
+        achieved = flops / (res["ms_step"] / 1e3) / 1e12
+        nbytes = recurrent_bytes(c)
+        t_roof = max(flops / (bf16_peak * 1e12), nbytes / (hbm * 1e9)) * 1e3
+        line["roofline"] = {
+            "kernel": "whole recurrent path (rehyat_step: %d steps x 4 kernels)" % (-(-c["F"] // c["T_c"])),
+            "bound": "tensor", "achieved": achieved, "peak": bf16_peak, "unit": "TFLOP/s",
+            "frac": achieved / bf16_peak, "peak_source": f"{src} bf16 dense (burst)",
+            "frac_of_sustained": achieved / bf16_sus if bf16_sus else None, "traffic": None,
+            "flops_per_video": flops, "algorithmic_bytes": nbytes, "roofline_ms_per_video": t_roof,
+            "ms_per_video": res["ms_step"],
+        }
     line["clocks"] = res["clocks"]
     line["gpu_launches"] = res["launches"]
     if args.config != "recurrent" and (args.sets != "causal" or args.layout != "bhnd" or args.phi == "mlp"):
@@ -634,45 +666,82 @@ def run_compare_full(args):
 
 
 def run_sweep(args):
+    """Every (F, T_c, T_o) point of the scaling sweep (B=2, H=12, d=128, 1560
+    tokens a frame): the two stages timed apart with CUDA events over at least
+    50 iterations (and at least ~1 s of work), SM clocks sampled over the same
+    region, and the roofline fraction of each stage.  The linear fit of time
+    against F is given for the raw times and for the times scaled to the
+    maximum SM clock (time x median MHz / max MHz), so that a clock drop under
+    the power cap can be told apart from a growth of the work per frame."""
     import numpy as np
     import torch
     from linear_attention_video_chunk_b200 import inputs
     from linear_attention_video_chunk_b200 import rehyat as R
     dev = torch.device("cuda", 0)
-    bf16_peak, _, _, src = peaks()
+    bf16_peak, bf16_sus, hbm, src = peaks()
     B, H, d, S = 2, 12, 128, 1560
     res = {}
     for F, Tc, To in SWEEP:
         q, k, v = (x.to(dev) for x in inputs.make_qkv(B, H, F * S, d, 100 + len(res), rms_qk=True))
         out = torch.empty_like(q)
         ws = R.alloc_workspace(R.workspace_bytes(B, H, F, S, d, Tc, To), dev)
+
+        def step(e=None):
+            if e is not None:
+                e[0].record()
+            R.forward_states(k, v, F, S, Tc, To, ws)
+            if e is not None:
+                e[1].record()
+            R.forward_attention(q, k, v, F, S, Tc, To, out, ws)
+            if e is not None:
+                e[2].record()
+
         for _ in range(3):
-            R.forward(q, k, v, F, S, Tc, To, out=out, workspace=ws)
+            step()
         torch.cuda.synchronize()
-        K = 10
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record()
-        for _ in range(K):
-            R.forward(q, k, v, F, S, Tc, To, out=out, workspace=ws)
-        e1.record()
+        t0 = time.perf_counter()
+        step()
         torch.cuda.synchronize()
-        ms = e0.elapsed_time(e1) / K
+        est = max(time.perf_counter() - t0, 1e-4)
+        K = int(min(1000, max(50, 1.0 / est)))
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+        with ClockSampler(dev) as clk:
+            for i in range(K):
+                step(ev[i])
+            torch.cuda.synchronize()
+        ms = ev[0][0].elapsed_time(ev[-1][2]) / K
+        st_ms = statistics.median(e[0].elapsed_time(e[1]) for e in ev)
+        at_ms = statistics.median(e[1].elapsed_time(e[2]) for e in ev)
+        cl = clk.summary()
+        scale = (cl["sm_mhz"] / cl["sm_max_mhz"]) if cl["sm_mhz"] and cl["sm_max_mhz"] else float("nan")
         w = work(dict(B=B, H=H, d=d, F=F, S_tok=S, T_c=Tc, T_o=To))
-        frac = (w["attn_flops"] + w["state_flops"]) / (ms / 1e3) / 1e12 / bf16_peak
-        res[(F, Tc, To)] = ms
-        print(json.dumps({"sweep_point": {"B": B, "H": H, "F": F, "T_c": Tc, "T_o": To}, "ms": ms,
-                          "tokens_per_s": B * F * S / (ms / 1e3), "roofline_frac": frac,
-                          "peak": f"{bf16_peak} TFLOP/s {src}"}), flush=True)
+        res[(F, Tc, To)] = (ms, ms * scale)
+        print(json.dumps({
+            "sweep_point": {"B": B, "H": H, "F": F, "T_c": Tc, "T_o": To}, "steps": K, "ms": ms,
+            "ms_at_max_clock": ms * scale, "ms_per_frame": ms / F, "states_ms": st_ms, "attention_ms": at_ms,
+            "tokens_per_s": B * F * S / (ms / 1e3),
+            "roofline": {"kernel": "hybrid_chunk_attn_kernel", "bound": "tensor",
+                         "achieved": w["attn_flops"] / (at_ms / 1e3) / 1e12, "peak": bf16_peak,
+                         "unit": "TFLOP/s", "frac": w["attn_flops"] / (at_ms / 1e3) / 1e12 / bf16_peak,
+                         "frac_of_sustained": w["attn_flops"] / (at_ms / 1e3) / 1e12 / bf16_sus if bf16_sus else None,
+                         "peak_source": f"{src} bf16 dense (burst)"},
+            "states_roofline": {"bound": "hbm", "achieved": w["state_bytes"] / (st_ms / 1e3) / 1e9, "peak": hbm,
+                                "unit": "GB/s", "frac": w["state_bytes"] / (st_ms / 1e3) / 1e9 / hbm},
+            "path_frac": (w["attn_flops"] + w["state_flops"]) / (ms / 1e3) / 1e12 / bf16_peak,
+            "clocks": cl}), flush=True)
         del q, k, v, out, ws
         torch.cuda.empty_cache()
     for Tc, To in ((2, 1), (3, 1), (5, 2)):
         Fs = np.array([F for F, a, b in SWEEP if (a, b) == (Tc, To)], dtype=float)
-        ts = np.array([res[(F, Tc, To)] for F in Fs.astype(int)])
         A = np.stack([Fs, np.ones_like(Fs)], 1)
-        coef, *_ = np.linalg.lstsq(A, ts, rcond=None)
-        r2 = 1 - ((A @ coef - ts) ** 2).sum() / ((ts - ts.mean()) ** 2).sum()
-        print(json.dumps({"linear_fit": {"T_c": Tc, "T_o": To, "ms_per_frame": coef[0], "intercept_ms": coef[1],
-                                         "r2": r2}}), flush=True)
+        fit = {"T_c": Tc, "T_o": To}
+        for i, key in ((0, "raw"), (1, "at_max_clock")):
+            ts = np.array([res[(F, Tc, To)][i] for F in Fs.astype(int)])
+            coef, *_ = np.linalg.lstsq(A, ts, rcond=None)
+            r2 = 1 - ((A @ coef - ts) ** 2).sum() / ((ts - ts.mean()) ** 2).sum()
+            fit[key] = {"ms_per_frame": coef[0], "intercept_ms": coef[1], "r2": r2,
+                        "ms_per_frame_each_F": [round(t / F, 5) for t, F in zip(ts, Fs)]}
+        print(json.dumps({"linear_fit": fit}), flush=True)
 
 
 # --------------------------------------------------------------------------- #
@@ -739,8 +808,7 @@ def run_reference(args):
         "impl": "reference", "metric": METRIC, "value": val, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": sec * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic (same generator and seed as the GPU arm)",
-        "config": {"workload": c["workload"], "B": B, "H": H, "d": d, "F": F, "S_tok": S,
-                   "chunk_frames": c["T_c"], "overlap_frames": c["T_o"]},
+        "config": config_dict(c, world),
         "cpu_baseline": {"value": val, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
                          "sample": f"each step: fp64 explicit-mask oracle on {n} random query rows x all {H} heads"},
         "e2e": {"value": val, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
