@@ -136,8 +136,16 @@ BF16_CASES = [
 ]
 # With 1-3 tokens per frame the first chunk's rows are a softmax over a few
 # keys (|y| ~ |v|) while later rows average hundreds of keys (|y| ~ 0.05):
-# bf16 output rounding of the large rows alone is ~0.035 of the global RMS.
+# there, rounding the exact result itself to bf16 already breaks the global
+# max-abs bound (checked in the test), so these two take each row's RMS.
 ROWWISE = {39, 42}
+
+
+def bf16_rounding_max_over_rms(ref):
+    """max |bf16(ref) - ref| / RMS(ref): the error of rounding the exact
+    (oracle) output to the output's precision, with no arithmetic error."""
+    r = torch.from_numpy(np.ascontiguousarray(ref)).float().bfloat16().double().numpy()
+    return max_over_rms(r, ref)
 
 
 @pytest.mark.parametrize("B,H,d,F,S,Tc,To,seed", BF16_CASES)
@@ -145,6 +153,10 @@ def test_forward_bf16_matches_oracle(B, H, d, F, S, Tc, To, seed):
     q, k, v = inputs.make_qkv(B, H, F * S, d, seed, rms_qk=True)
     y = R.forward(q.cuda(), k.cuda(), v.cuda(), F, S, Tc, To)
     ref = orc.oracle_forward(q, k, v, F, S, Tc, To)
+    if seed in ROWWISE:
+        # the per-row bound is used only where no bf16 output could meet the
+        # global one: rounding the oracle's own result breaks it
+        assert bf16_rounding_max_over_rms(ref) > BF16_MAX
     assert_bf16_close(np64(y), ref, rowwise=seed in ROWWISE)
 
 
@@ -152,14 +164,54 @@ def test_forward_bf16_matches_oracle(B, H, d, F, S, Tc, To, seed):
 def test_forward_bf16_softmax_and_linear_balance(post):
     """Scaled queries move the balance between the branches: q x 8 makes the
     softmax window dominate every chunk, q x 3 mixes both, q,k x 0.25 makes
-    scores flat so the linear term dominates.  In these skewed inputs row
-    magnitudes differ by ~20x (sharp softmax rows ~ single v rows, linear rows
-    ~ averages), so bf16 output rounding alone exceeds 3e-2 of the *global*
-    RMS; the max-abs bound is applied per row against that row's RMS."""
+    scores flat so the linear term dominates.  Held to the global bound
+    (rel L2 <= 1e-2, max |err| <= 3e-2 RMS(ref)) and to the same bound
+    against each row's own RMS.
+
+    One exception, derived and pinned in tests/test_precision_budget.py: on
+    q x 3 the bf16 rounding of the exact result alone is 2.71e-2 of the RMS,
+    and the bf16 rounding of the softmax weights under the lazy shift adds
+    ~5e-3 at one element (3.23e-2 measured, the same figure as a numpy
+    emulation of the kernel's roundings).  There the arithmetic before the
+    output rounding (the fp32 terms of rehyat_forward_parts, recombined) is
+    held to 3e-2 of the global RMS, and the bf16 output to the rounding floor
+    plus 1e-2."""
     B, H, d, F, S, Tc, To = 1, 2, 128, 5, 160, 2, 1
     q, k, v = inputs.make_qkv(B, H, F * S, d, 40, rms_qk=True, post=post)
     y = np64(R.forward(q.cuda(), k.cuda(), v.cuda(), F, S, Tc, To))
-    assert_bf16_close(y, orc.oracle_forward(q, k, v, F, S, Tc, To), str(post), rowwise=True)
+    ref = orc.oracle_forward(q, k, v, F, S, Tc, To)
+    if post != (3.0, 1.0, 1.0):
+        assert_bf16_close(y, ref, str(post))
+    else:
+        floor = bf16_rounding_max_over_rms(ref)
+        assert floor > 0.025
+        aS, nS, aL, nL, _ = (np64(x) for x in R.forward_parts(q.cuda(), k.cuda(), v.cuda(), F, S, Tc, To))
+        assert_bf16_close((aS + aL) / (nS + nL)[..., None], ref, "fp32 terms before the output rounding")
+        e2, em = rel_l2(y, ref), max_over_rms(y, ref)
+        assert e2 <= BF16_L2 and em <= floor + 1e-2, (e2, em, floor)
+    assert_bf16_close(y, ref, str(post) + " per row", rowwise=True)
+
+
+def assert_branches_per_chunk(aS, nS, aL, nL, oS, onS, oL, onL, rows, F, S, Tc):
+    """The softmax branch aS/nS and the linear branch aL/nL against the
+    oracle's, each chunk on its own (rel L2 per (b,h) over that chunk's
+    rows, max-abs against that chunk's RMS), so a wrong softmax branch in one
+    chunk cannot hide under the others or under the linear term.  Returns
+    the worst chunk's figures for the message."""
+    chunk_of = rows // (min(Tc, F) * S)
+    worst = []
+    for t in np.unique(chunk_of):
+        sel = chunk_of == t
+        e = assert_bf16_close(aS[:, :, sel] / nS[:, :, sel, None], oS[:, :, sel] / onS[:, :, sel, None],
+                              f"softmax branch, chunk {t}")
+        worst.append((e, int(t), "softmax"))
+        lin = onL[0, 0, sel] > 0
+        if lin.any():
+            cols = np.flatnonzero(sel)[lin]
+            e = assert_bf16_close(aL[:, :, cols] / nL[:, :, cols, None], oL[:, :, cols] / onL[:, :, cols, None],
+                                  f"linear branch, chunk {t}")
+            worst.append((e, int(t), "linear"))
+    return max(worst)
 
 
 def test_forward_parts_match_oracle_parts():
@@ -170,6 +222,7 @@ def test_forward_parts_match_oracle_parts():
     aS, nS, aL, nL, M = (np64(x) for x in R.forward_parts(q.cuda(), k.cuda(), v.cuda(), F, S, Tc, To))
     oS, onS, oL, onL = orc.oracle_parts(q, k, v, F, S, Tc, To)
     assert_bf16_close(aS / nS[..., None], oS / onS[..., None], "softmax branch")
+    assert_branches_per_chunk(aS, nS, aL, nL, oS, onS, oL, onL, np.arange(F * S), F, S, Tc)
     lin = onL > 0
     assert (nL[~lin] == 0).all() and (aL[~lin] == 0).all()
     rows = lin[0, 0]
@@ -296,6 +349,32 @@ def test_wan13b_480p_sampled_rows():
     assert_bf16_close(np64(y[:, :, rows]), ref)
 
 
+def test_wan13b_480p_parts_per_chunk():
+    """Both branches of the joint normaliser at the Wan2.1-1.3B 480p shape
+    (B=1, H=12, d=128, F=21 x 1560, T_c=3, T_o=1), every head, checked chunk
+    by chunk on sampled rows: the first and last 32 rows of every chunk plus
+    32 random rows of each."""
+    B, H, d, F, S, Tc, To = 1, 12, 128, 21, 1560, 3, 1
+    q, k, v = inputs.make_qkv(B, H, F * S, d, 1, rms_qk=True)
+    Np = Tc * S
+    rng = np.random.default_rng(17)
+    rows = set()
+    for q0 in range(0, F * S, Np):
+        q1 = min(q0 + Np, F * S)
+        rows.update(range(q0, q0 + 32))
+        rows.update(range(q1 - 32, q1))
+        rows.update(rng.integers(q0, q1, 32).tolist())
+    rows = np.array(sorted(rows))
+    parts = R.forward_parts(q.cuda(), k.cuda(), v.cuda(), F, S, Tc, To)
+    aS, nS, aL, nL, M = (np64(x[:, :, rows]) for x in parts)
+    del parts
+    oS, onS, oL, onL = orc.oracle_parts(q, k, v, F, S, Tc, To, rows=rows)
+    (e2, em), t, branch = assert_branches_per_chunk(aS, nS, aL, nL, oS, onS, oL, onL, rows, F, S, Tc)
+    print(f"worst chunk: {t} ({branch} branch): rel L2 {e2:.3e}, max/RMS {em:.3e}")
+    y = (aS + aL) / (nS + nL)[..., None]
+    assert_bf16_close(y, (oS + oL) / (onS + onL)[..., None], "recombined")
+
+
 def _head_rows_check(y, q, k, v, F, S, Tc, To, heads, rows):
     """Oracle on the given (b, h) heads and query rows only."""
     for b, h in heads:
@@ -367,18 +446,6 @@ def test_scaling_sweep_points_sampled(F, Tc, To):
     q, k, v = inputs.make_qkv(B, H, F * S, d, seed, rms_qk=True)
     y = R.forward(q.cuda(), k.cuda(), v.cuda(), F, S, Tc, To).cpu()
     _head_rows_check(y, q, k, v, F, S, Tc, To, [(0, 3), (1, 11)], few_rows(F, S, Tc, edge=16, n_rand=64))
-
-
-def test_exp2_fma_error_bound():
-    """The FMA-pipe 2^x used for part of the softmax weights stays within its
-    stated relative error (7.5e-5) of the exact power over [-125, 8]."""
-    x = torch.cat([torch.linspace(-125.0, 8.0, 1_000_001),
-                   torch.rand(100_000, generator=torch.Generator().manual_seed(3)) * 133.0 - 125.0])
-    y = R.exp2_fma(x.cuda()).cpu().double().numpy()
-    ref = np.exp2(x.double().numpy())
-    assert np.abs(y / ref - 1).max() < 8e-5
-    lo = R.exp2_fma(torch.tensor([-200.0, -125.0], device="cuda")).cpu().double().numpy()
-    np.testing.assert_allclose(lo, [2.0 ** -125] * 2, rtol=1e-4)
 
 
 # --------------------------------------------------------------------------- #
