@@ -306,7 +306,10 @@ int rehyat_chunk_states(const void* k, const void* v,
  *     before launching anything (1.3B-480p needs ~30 MB and fits).
  *   - The first call on a device looks up the array's device address
  *     (cudaGetSymbolAddress, with that device current); make that first call
- *     before any stream capture.
+ *     before any stream capture.  Later calls made outside stream capture
+ *     look it up again, so after a cudaDeviceReset the next ordinary call
+ *     uses the reloaded array; calls recorded into a stream capture use the
+ *     address of the last lookup on that device.
  *   - All calls on a device share the one array: calls whose kernels overlap
  *     on the GPU (different streams, no ordering) race and corrupt each
  *     other; order them.  Each call writes every scratch byte it reads. */
@@ -373,13 +376,6 @@ int rehyat_step_f32(const float* q_c, const float* k_c, const float* v_c,
  * bad sizes. */
 int rehyat_phi(const void* x, int x_dtype, void* y, int y_dtype,
                int64_t rows, int d, void* stream);
-
-/* Diagnostic: y[i] = 2^x[i] by the FMA-pipe exponential the fused kernel uses
- * for part of its softmax weights (round-to-nearest range reduction and a
- * fitted cubic; max relative error 7.5e-5 for x in [-125, 8]; x < -125 is
- * treated as -125).  x, y: n floats in device memory (4-byte aligned);
- * REHYAT_EINVAL for null / misaligned pointers or n < 1. */
-int rehyat_exp2_fma(const float* x, float* y, int64_t n, void* stream);
 
 /* Diagnostic for the failure path: launches one warp that waits on a
  * barrier nothing ever completes.  The wait is bounded like every device

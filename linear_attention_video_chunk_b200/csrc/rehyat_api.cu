@@ -1008,12 +1008,6 @@ REHYAT_API int rehyat_phi(const void* x, int x_dtype, void* y, int y_dtype, int6
                                 static_cast<cudaStream_t>(stream)));
 }
 
-REHYAT_API int rehyat_exp2_fma(const float* x, float* y, int64_t n, void* stream) {
-  if (x == nullptr || y == nullptr || n < 1) return REHYAT_EINVAL;
-  if (reinterpret_cast<uintptr_t>(x) % 4 != 0 || reinterpret_cast<uintptr_t>(y) % 4 != 0) return REHYAT_EINVAL;
-  return cuda_status(launch_exp2_fma(x, y, n, static_cast<cudaStream_t>(stream)));
-}
-
 REHYAT_API int rehyat_wait_probe(int* gave_up, void* stream) {
   return cuda_status(launch_wait_probe(gave_up, static_cast<cudaStream_t>(stream)));
 }
@@ -1043,8 +1037,12 @@ REHYAT_API int rehyat_device_status(unsigned int* detail) {
 //
 // In host code the name g_noalloc_scratch is only a host-side stand-in for
 // the device array, never a device address; the address is looked up with
-// cudaGetSymbolAddress once per device (on that device's first call, with the
-// device current) and only that address is handed to kernels and to TMA.
+// cudaGetSymbolAddress with the device current (first on that device's first
+// call) and only that address is handed to kernels and to TMA.  Every call
+// made outside stream capture looks it up again, so a device reset (which
+// reloads the module, possibly at another address) is picked up by the next
+// ordinary call; while a stream is being captured the address of the last
+// lookup on that device is used.
 namespace {
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[REHYAT_NOALLOC_SCRATCH_BYTES];
@@ -1054,11 +1052,16 @@ std::mutex g_noalloc_mu;
 void* g_noalloc_addr[kMaxDevices] = {};
 
 // Device address of the scratch array on the current device.
-int noalloc_scratch(void** addr) {
+int noalloc_scratch(cudaStream_t s, void** addr) {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return REHYAT_ECUDA;
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(s, &cap) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return REHYAT_ECUDA;
+  }
   std::lock_guard<std::mutex> lock(g_noalloc_mu);
-  if (g_noalloc_addr[dev] == nullptr) {
+  if (cap == cudaStreamCaptureStatusNone || g_noalloc_addr[dev] == nullptr) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) {
       (void)cudaGetLastError();
@@ -1098,12 +1101,12 @@ REHYAT_API int rehyat_forward_noalloc(const void* q, const void* k, const void* 
   int nsplit = P.nsplit;
   while (layout_with_nsplit(&P, nsplit) > REHYAT_NOALLOC_SCRATCH_BYTES && nsplit > 1) --nsplit;
   if (P.bytes > REHYAT_NOALLOC_SCRATCH_BYTES) return REHYAT_ENOMEM;  // problem too large for the array
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
   void* ws = nullptr;
-  st = noalloc_scratch(&ws);
+  st = noalloc_scratch(s, &ws);
   if (st != REHYAT_OK) return st;
   // Every scratch byte this call reads is first written by this call, so
   // nothing is cleared; calls that overlap on the GPU share the array and race.
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
   uint8_t* w = static_cast<uint8_t*>(ws);
   st = run_states(k, v, P, w, nullptr, nullptr, s);
   if (st != REHYAT_OK) return st;

@@ -39,8 +39,8 @@ def _close(y, ref):
 def test_noalloc_matches_forward_on_two_calls_in_a_row():
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
-    # the Wan2.1-1.3B 480p shape: its scratch (~30 MB once pieces are merged)
-    # fits the 32 MiB array
+    # the Wan2.1-1.3B 480p shape: its default scratch layout (~30 MB) fits
+    # the 32 MiB array as it is
     B, H, d, F, S, Tc, To = 1, 12, 128, 21, 1560, 3, 1
     L = R.lib()
     for seed in (1, 5):
@@ -57,6 +57,30 @@ def test_noalloc_matches_forward_on_two_calls_in_a_row():
         if R.workspace_bytes(B, H, F, S, d, Tc, To) <= R.NOALLOC_SCRATCH_BYTES:
             # same scratch layout as rehyat_forward: same kernels, same order
             assert torch.equal(out, ref)
+    assert R.device_status() == R.OK
+
+
+def test_noalloc_merges_key_pieces_when_the_default_layout_does_not_fit():
+    """B=1, H=37, d=128, F=9 x 64 tokens, T_c=3, T_o=1: the default layout
+    sums each key segment in two pieces (~34 MB of scratch, more than the
+    array); the array version sums them in one piece (~24 MB), so its result
+    differs from rehyat_forward's only by fp32 summation order."""
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    B, H, d, F, S, Tc, To = 1, 37, 128, 9, 64, 3, 1
+    assert R.workspace_bytes(B, H, F, S, d, Tc, To) > R.NOALLOC_SCRATCH_BYTES
+    L = R.lib()
+    for seed in (6, 7):
+        q, k, v = (x.cuda() for x in inputs.make_qkv(B, H, F * S, d, seed, rms_qk=True))
+        ref = R.forward_capi(q, k, v, F, S, Tc, To)
+        out = torch.full_like(q, float("nan"))
+        st = L.rehyat_forward_noalloc(q.data_ptr(), k.data_ptr(), v.data_ptr(), B, H, F, S, d, Tc, To,
+                                      out.data_ptr(), ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+        assert st == R.OK, R.status_string(st)
+        torch.cuda.synchronize()
+        assert torch.isfinite(out.float()).all()
+        e2, em = _close(out, ref)
+        assert e2 <= BF16_L2 and em <= BF16_MAX, (seed, e2, em)
     assert R.device_status() == R.OK
 
 
