@@ -130,7 +130,6 @@ cudaError_t launch_state_split(const float* S, long long n, __nv_bfloat16* hi, _
                                cudaStream_t s);
 
 // The FMA-pipe exp2 used for part of the softmax exponentials (diagnostic).
-cudaError_t launch_exp2_fma(const float* x, float* y, long long n, cudaStream_t s);
 
 cudaError_t launch_attention_f32(const AttnF32Params& p, int n_chunks, cudaStream_t s);
 cudaError_t launch_chunk_state_f32(const StateF32Params& p, cudaStream_t s);

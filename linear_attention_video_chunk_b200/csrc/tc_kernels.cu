@@ -20,34 +20,10 @@
 namespace rehyat {
 namespace {
 
-// 2^x on the FMA/ALU pipes, for the share of softmax exponentials taken off
-// the SFU.  Range reduction: n = round(x) by adding 1.5 * 2^23 (the rounding
-// happens in the fp32 add), f = x - n in [-0.5, 0.5]; 2^f by a cubic whose
-// coefficients were fitted here to minimise relative error (Chebyshev-node
-// least squares with Lawson reweighting); n is then added to the result's
-// exponent field.  Max relative error in fp32 over [-125, 8]: 7.5e-5, far
-// below the 2^-9 of the bf16 P it feeds.  x < -125 is clamped (2^-125 stands
-// in for ~0); callers never pass -inf.
-__device__ __forceinline__ float exp2_fma(float x) {
-  x = fmaxf(x, -125.f);
-  const float t = x + 12582912.f;
-  const float f = x - (t - 12582912.f);
-  const float p = fmaf(fmaf(fmaf(0x1.c3f748p-5f, f, 0x1.f0de1ap-3f), f, 0x1.62f31ap-1f), f, 0x1.fff692p-1f);
-  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
-}
-
-#ifndef REHYAT_EXP2_FMA_MASK
-// Columns c of each score tile with bit (c % 8) set take exp2_fma instead
-// of ex2 (0x11 = 2 of 8).  Measured on B200 at the Wan2.1-1.3B shape, any
-// share made the kernel slower (the softmax is latency-bound, not SFU-bound),
-// so the default is none.
-#define REHYAT_EXP2_FMA_MASK 0x00u
-#endif
-
 // P = 2^(s * scale - m) for one half (64 keys) of a 128-key row tile, packed
 // to bf16 pairs and stored into TMEM columns [32*HALF, 32*HALF + 32) of S;
 // returns the row sum of exactly the stored bf16 values.
-template <uint32_t FMA_MASK, int HALF>
+template <int HALF>
 __device__ __forceinline__ float exp_pack_store(uint32_t (&s)[4][32], float scale, float neg_m, uint32_t tS) {
   float rsum[4] = {0.f, 0.f, 0.f, 0.f};  // independent partial sums
   uint32_t pk[32];
@@ -60,8 +36,8 @@ __device__ __forceinline__ float exp_pack_store(uint32_t (&s)[4][32], float scal
       // 2% faster for the whole kernel than two scalar FMAs)
       float x0, x1;
       fma_f32x2(s[a][2 * c], s[a][2 * c + 1], sc2, nm2, x0, x1);
-      const float p0 = ((FMA_MASK >> ((2 * c) & 7)) & 1u) ? exp2_fma(x0) : ex2(x0);
-      const float p1 = ((FMA_MASK >> ((2 * c + 1) & 7)) & 1u) ? exp2_fma(x1) : ex2(x1);
+      const float p0 = ex2(x0);
+      const float p1 = ex2(x1);
       const uint32_t u = pack_bf16(p0, p1);
       // the denominator sums exactly the bf16 weights the P.V MMA uses
       float& acc = rsum[c & 3];
@@ -273,11 +249,9 @@ __global__ void __launch_bounds__(384, 1) hybrid_chunk_attn_kernel(const __grid_
         m_used = mnew;
         const float neg_m = -m_used;
         // P is released in two 64-key halves, so the first half's P.V runs
-        // on the tensor core while the second half's exponentials are taken.
-        // Full tiles may send a share of the exponentials to the FMA pipe;
-        // the window's partial last tile stays on ex2 (masked keys give 0).
-        float rs = (valid >= 128) ? exp_pack_store<REHYAT_EXP2_FMA_MASK, 0>(s, p.scale_log2, neg_m, tS)
-                                  : exp_pack_store<0u, 0>(s, p.scale_log2, neg_m, tS);
+        // on the tensor core while the second half's exponentials are taken
+        // (masked keys of the window's partial last tile give 0).
+        float rs = exp_pack_store<0>(s, p.scale_log2, neg_m, tS);
         if (warp_need && j > 0) {
           // O holds tiles 0..j-1 (their P.V completed before S_j was
           // signalled) and must move to the new shift before P_j.V_j.
@@ -296,8 +270,7 @@ __global__ void __launch_bounds__(384, 1) hybrid_chunk_attn_kernel(const __grid_
         }
         warp_release(BAR(C::B_P + X), lane);
         if (wl == 0 && lane == 0) TRACE(3 + 5 * X, j);
-        rs += (valid >= 128) ? exp_pack_store<REHYAT_EXP2_FMA_MASK, 1>(s, p.scale_log2, neg_m, tS)
-                             : exp_pack_store<0u, 1>(s, p.scale_log2, neg_m, tS);
+        rs += exp_pack_store<1>(s, p.scale_log2, neg_m, tS);
         warp_release(BAR(C::B_P1 + X), lane);
         if (wl == 0 && lane == 0) TRACE(4 + 5 * X, j);
         l = l * alpha + rs;
@@ -616,18 +589,6 @@ __global__ void __launch_bounds__(384, 1) hybrid_chunk_attn_kernel(const __grid_
   }
 }
 
-__global__ void exp2_fma_kernel(const float* __restrict__ x, float* __restrict__ y, long long n) {
-  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n;
-       i += static_cast<long long>(gridDim.x) * blockDim.x)
-    y[i] = exp2_fma(x[i]);
-}
-
-int grid_for(long long n, int threads) {
-  long long g = (n + threads - 1) / threads;
-  if (g > 148LL * 16) g = 148LL * 16;
-  return static_cast<int>(g < 1 ? 1 : g);
-}
-
 }  // namespace
 
 int attn_smem_bytes(int D) { return D == 128 ? AttnCfg<128>::SMEM : AttnCfg<64>::SMEM; }
@@ -653,11 +614,6 @@ cudaError_t launch_attention(int D, bool parts, const AttnParams& p, int n_units
 cudaError_t launch_attention_phi(int D, const AttnParams& p, int n_units, cudaStream_t s) {
   if (n_units <= 0) return cudaSuccess;
   return D == 128 ? launch_attn_t<128, false, true>(p, n_units, s) : launch_attn_t<64, false, true>(p, n_units, s);
-}
-
-cudaError_t launch_exp2_fma(const float* x, float* y, long long n, cudaStream_t s) {
-  exp2_fma_kernel<<<grid_for(n, 256), 256, 0, s>>>(x, y, n);
-  return cudaGetLastError();
 }
 
 }  // namespace rehyat

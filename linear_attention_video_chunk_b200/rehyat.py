@@ -36,7 +36,6 @@ _SIGS = {
     "rehyat_phi": [_vp, _I, _vp, _I, ctypes.c_int64, _I, _vp],
     "rehyat_device_status": [ctypes.POINTER(ctypes.c_uint)],
     "rehyat_forward_noalloc": [_vp, _vp, _vp, _I, _I, _I, _I, _I, _I, _I, _vp, _vp],
-    "rehyat_exp2_fma": [_vp, _vp, ctypes.c_int64, _vp],
     "rehyat_forward_ex_workspace_bytes": [_I, _I, _I, _I, _I, _I, _I, _I, ctypes.POINTER(_c_size)],
     "rehyat_forward_ex": [_vp, _vp, _vp, _I, _I, _I, _I, _I, _I, _I, _I, _I, _vp, _vp, _c_size, _vp],
     "rehyat_phi_mlp": [_vp, _I, _I, _I, _I, _I, _vp, _vp, _vp, _vp, _vp, _vp],
@@ -494,14 +493,6 @@ def phi(x: torch.Tensor, out_dtype=None) -> torch.Tensor:
     y = torch.empty(*x.shape[:-1], 2 * d, dtype=od, device=x.device)
     code = lambda dt: DTYPE_BF16 if dt == torch.bfloat16 else DTYPE_F32
     _check(lib().rehyat_phi(_p(x), code(x.dtype), _p(y), code(od), rows, d, _stream()), "rehyat_phi")
-    return y
-
-
-def exp2_fma(x: torch.Tensor) -> torch.Tensor:
-    """The fused kernel's FMA-pipe 2^x (diagnostic), on a CUDA float tensor."""
-    _need(x, torch.float32, "x", x.dim())
-    y = torch.empty_like(x)
-    _check(lib().rehyat_exp2_fma(_p(x), _p(y), x.numel(), _stream()), "rehyat_exp2_fma")
     return y
 
 

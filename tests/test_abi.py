@@ -320,8 +320,6 @@ def test_elementwise_calls_check_element_alignment(lib):
     assert lib.rehyat_phi(0x10001, 0, 0x10000, 0, 4, 64, None) == R.EINVAL       # bf16 x at an odd address
     assert lib.rehyat_phi(0x10000, 1, 0x10002, 1, 4, 64, None) == R.EINVAL       # fp32 y at 2 mod 4
     assert lib.rehyat_phi(0x10000, 2, 0x10000, 0, 4, 64, None) == R.EINVAL       # unknown dtype
-    assert lib.rehyat_exp2_fma(0x10002, 0x10000, 4, None) == R.EINVAL
-    assert lib.rehyat_exp2_fma(0x10000, 0x10000, 0, None) == R.EINVAL
 
 
 _BAD_SIZES = dict(B=[0, -1], H=[0], F=[0], S_tok=[0], N=[0], d=[96, 0], chunk_frames=[0], overlap_frames=[-1],
