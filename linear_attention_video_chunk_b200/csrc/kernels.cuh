@@ -103,16 +103,36 @@ inline cudaError_t prepare_kernel_once(const void* func, int smem, int need_regs
   return e;
 }
 
+// Launch `k` on stream s; with pdl the launch carries a programmatic
+// dependency on the previous kernel in the stream, so its CTAs may be
+// scheduled before that kernel has finished (the kernel itself waits, with
+// griddepcontrol.wait, before touching what the previous kernel writes).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_k(void (*k)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, bool pdl,
+                     Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, k, std::forward<Args>(args)...);
+}
+
 // Shared-memory bytes each tensor-core kernel needs (dynamic).
 int attn_smem_bytes(int D);
 int state_smem_bytes(int D);
 
-cudaError_t launch_attention(int D, bool parts, const AttnParams& p, int n_units, cudaStream_t s);
-cudaError_t launch_chunk_state(int D, const StateParams& p, int n_ctas, cudaStream_t s);
+cudaError_t launch_attention(int D, bool parts, const AttnParams& p, int n_units, cudaStream_t s, bool pdl = false);
+cudaError_t launch_chunk_state(int D, const StateParams& p, int n_ctas, cudaStream_t s, bool pdl = false);
 // Variants reading precomputed feature maps: phi(K) through p.tm_phik (the
 // states) and phi(Q) rows from p.phi_q (the attention epilogue).
-cudaError_t launch_attention_phi(int D, const AttnParams& p, int n_units, cudaStream_t s);
-cudaError_t launch_chunk_state_phi(int D, const StateParams& p, int n_ctas, cudaStream_t s);
+cudaError_t launch_attention_phi(int D, const AttnParams& p, int n_units, cudaStream_t s, bool pdl = false);
+cudaError_t launch_chunk_state_phi(int D, const StateParams& p, int n_ctas, cudaStream_t s, bool pdl = false);
 // Exclusive prefix over segments (and sum over pieces): writes the state
 // entering each chunk, either as bf16 hi/lo (hi, lo non-null) or fp32 (Sf).
 cudaError_t launch_state_scan(const float* part_S, const float* part_z, int BH, int n_seg,
@@ -124,7 +144,7 @@ cudaError_t launch_state_scan_bidir(const float* part_S, const float* part_z, in
                                     float* Sf, float* zt, cudaStream_t s);
 // state_S/z += sum over pieces of one segment's partials.
 cudaError_t launch_state_accumulate(const float* part_S, const float* part_z, int BH, int nsplit,
-                                    int D, float* state_S, float* state_z, cudaStream_t s);
+                                    int D, float* state_S, float* state_z, cudaStream_t s, bool pdl = false);
 // fp32 state -> bf16 hi/lo pair.
 cudaError_t launch_state_split(const float* S, long long n, __nv_bfloat16* hi, __nv_bfloat16* lo,
                                cudaStream_t s);

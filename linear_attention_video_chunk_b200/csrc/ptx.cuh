@@ -79,6 +79,15 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
 }
 
 // ----------------------------------------------------------------------------
+// Programmatic dependent launch.  grid_dep_wait: wait until the grids this
+// grid depends on have completed and their memory is visible (returns at
+// once when the grid was launched without a programmatic dependency).
+// grid_dep_launch: this CTA lets the next grid in the stream be scheduled.
+// ----------------------------------------------------------------------------
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+// ----------------------------------------------------------------------------
 // TMA (bulk tensor copies, global -> shared, completion on an mbarrier)
 // ----------------------------------------------------------------------------
 __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, uint32_t bar,

@@ -853,11 +853,17 @@ int run_step(const void* q_c, const void* k_c, const void* v_c, const void* phi_
   ap.z_bh = 2LL * P.D;
   ap.z_t = 0;
   ap.out = static_cast<__nv_bfloat16*>(out_c);
+  // The attention, the fold of the evicted keys and the state update each
+  // follow the previous kernel with a programmatic dependency: the fold
+  // (which reads only this chunk's keys and values) fills the SMs the
+  // attention's last wave leaves idle; each kernel waits before it touches
+  // what an earlier one writes (the attention before its state tiles, the
+  // update before everything).
   if (phi_q != nullptr) {
     ap.phi_q = static_cast<const __nv_bfloat16*>(phi_q);
-    st = cuda_status(launch_attention_phi(P.D, ap, P.n_units, s));
+    st = cuda_status(launch_attention_phi(P.D, ap, P.n_units, s, true));
   } else {
-    st = cuda_status(launch_attention(P.D, false, ap, P.n_units, s));
+    st = cuda_status(launch_attention(P.D, false, ap, P.n_units, s, true));
   }
   if (st != REHYAT_OK || P.evict_tok == 0) return st;
   StateParams sp;
@@ -871,10 +877,10 @@ int run_step(const void* q_c, const void* k_c, const void* v_c, const void* phi_
   sp.H = P.H;
   sp.part_S = reinterpret_cast<float*>(w + P.off_pS);
   sp.part_z = reinterpret_cast<float*>(w + P.off_pz);
-  st = cuda_status(phi_k != nullptr ? launch_chunk_state_phi(P.D, sp, P.BH * P.nsplit, s)
-                                    : launch_chunk_state(P.D, sp, P.BH * P.nsplit, s));
+  st = cuda_status(phi_k != nullptr ? launch_chunk_state_phi(P.D, sp, P.BH * P.nsplit, s, true)
+                                    : launch_chunk_state(P.D, sp, P.BH * P.nsplit, s, true));
   if (st != REHYAT_OK) return st;
-  return cuda_status(launch_state_accumulate(sp.part_S, sp.part_z, P.BH, P.nsplit, P.D, state_S, state_z, s));
+  return cuda_status(launch_state_accumulate(sp.part_S, sp.part_z, P.BH, P.nsplit, P.D, state_S, state_z, s, true));
 }
 }  // namespace
 

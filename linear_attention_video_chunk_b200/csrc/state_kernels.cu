@@ -97,6 +97,10 @@ __global__ void state_scan_bidir_kernel(const float* __restrict__ pS, const floa
 
 __global__ void state_accumulate_kernel(const float* __restrict__ pS, const float* __restrict__ pz, int BH,
                                         int nsplit, int D, float* S, float* z) {
+  // In the recurrent step this kernel follows the fold of evicted keys with
+  // a programmatic dependency: wait until that fold (and so the attention
+  // before it, which reads z) has completed.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int W = D + 1;
   const long long total = static_cast<long long>(BH) * 2 * D * W;
   for (long long idx = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; idx < total;
@@ -154,10 +158,10 @@ cudaError_t launch_state_scan_bidir(const float* part_S, const float* part_z, in
 }
 
 cudaError_t launch_state_accumulate(const float* part_S, const float* part_z, int BH, int nsplit, int D,
-                                    float* state_S, float* state_z, cudaStream_t s) {
+                                    float* state_S, float* state_z, cudaStream_t s, bool pdl) {
   const long long n = static_cast<long long>(BH) * 2 * D * (D + 1);
-  state_accumulate_kernel<<<grid_for(n, 256), 256, 0, s>>>(part_S, part_z, BH, nsplit, D, state_S, state_z);
-  return cudaGetLastError();
+  return launch_k(state_accumulate_kernel, dim3(grid_for(n, 256)), dim3(256), 0, s, pdl, part_S, part_z, BH, nsplit,
+                  D, state_S, state_z);
 }
 
 cudaError_t launch_state_split(const float* S, long long n, __nv_bfloat16* hi, __nv_bfloat16* lo,

@@ -57,6 +57,7 @@ __global__ void __launch_bounds__(StCfg<D>::THREADS, 1) phi_state_kernel(const _
                                              ~static_cast<uintptr_t>(1023));
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  grid_dep_launch();  // the recurrent step's state update may be scheduled
   const int u = blockIdx.x;  // (bh * n_seg + s) * nsplit + piece
   const int piece = u % p.sg.nsplit;
   const int s = (u / p.sg.nsplit) % p.sg.n_seg;
@@ -69,6 +70,7 @@ __global__ void __launch_bounds__(StCfg<D>::THREADS, 1) phi_state_kernel(const _
   if (ntiles == 0) {  // empty piece: its sums are zero
     for (int i = threadIdx.x; i < 2 * D * D; i += blockDim.x) outS[i] = 0.f;
     for (int i = threadIdx.x; i < 2 * D; i += blockDim.x) outz[i] = 0.f;
+    grid_dep_wait();
     return;
   }
 
@@ -275,6 +277,11 @@ __global__ void __launch_bounds__(StCfg<D>::THREADS, 1) phi_state_kernel(const _
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
   }
+  // Launched behind the recurrent step's attention with a programmatic
+  // dependency (it reads only the chunk's keys and values): it completes only
+  // after that attention has, so the state update launched next may rely on
+  // both.  Launched normally, this returns at once.
+  grid_dep_wait();
 }
 
 // Failure-path check: one warp waits on an mbarrier that nothing ever
@@ -304,22 +311,21 @@ cudaError_t launch_wait_probe(int* gave_up, cudaStream_t s) {
 int state_smem_bytes(int D) { return D == 128 ? StCfg<128>::SMEM : StCfg<64>::SMEM; }
 
 template <int D, bool PRE = false>
-static cudaError_t launch_state_t(const StateParams& p, int n_ctas, cudaStream_t s) {
+static cudaError_t launch_state_t(const StateParams& p, int n_ctas, cudaStream_t s, bool pdl) {
   auto* k = phi_state_kernel<D, PRE>;
   cudaError_t e = prepare_kernel_once(reinterpret_cast<const void*>(k), StCfg<D>::SMEM, 0);
   if (e != cudaSuccess) return e;
-  k<<<n_ctas, StCfg<D>::THREADS, StCfg<D>::SMEM, s>>>(p);
-  return cudaGetLastError();
+  return launch_k(k, dim3(n_ctas), dim3(StCfg<D>::THREADS), StCfg<D>::SMEM, s, pdl, p);
 }
 
-cudaError_t launch_chunk_state(int D, const StateParams& p, int n_ctas, cudaStream_t s) {
+cudaError_t launch_chunk_state(int D, const StateParams& p, int n_ctas, cudaStream_t s, bool pdl) {
   if (n_ctas <= 0) return cudaSuccess;
-  return D == 128 ? launch_state_t<128>(p, n_ctas, s) : launch_state_t<64>(p, n_ctas, s);
+  return D == 128 ? launch_state_t<128>(p, n_ctas, s, pdl) : launch_state_t<64>(p, n_ctas, s, pdl);
 }
 
-cudaError_t launch_chunk_state_phi(int D, const StateParams& p, int n_ctas, cudaStream_t s) {
+cudaError_t launch_chunk_state_phi(int D, const StateParams& p, int n_ctas, cudaStream_t s, bool pdl) {
   if (n_ctas <= 0) return cudaSuccess;
-  return D == 128 ? launch_state_t<128, true>(p, n_ctas, s) : launch_state_t<64, true>(p, n_ctas, s);
+  return D == 128 ? launch_state_t<128, true>(p, n_ctas, s, pdl) : launch_state_t<64, true>(p, n_ctas, s, pdl);
 }
 
 cudaError_t read_and_clear_device_error_states(unsigned int* v) {

@@ -74,7 +74,8 @@ struct AttnCfg {
   static constexpr int B_O = B_P1 + 2;           // [2] last P.V done
   static constexpr int B_PHI = B_O + 2;          // [2] scaled phi(Q) written to TMEM
   static constexpr int B_LIN = B_PHI + 2;        // [2] linear MMA done
-  static constexpr int B_FIN = B_LIN + 2;        // MMA drain
+  static constexpr int B_PVD = B_LIN + 2;        // [2] P.V of the current key tile done
+  static constexpr int B_FIN = B_PVD + 2;        // MMA drain
   static constexpr int NBARS = B_FIN + 1;
   static_assert(NBARS * 8 <= 256, "barrier area");
   static_assert(SMEM <= 232448, "shared memory");
@@ -110,6 +111,10 @@ __global__ void __launch_bounds__(384, 1) hybrid_chunk_attn_kernel(const __grid_
                                              ~static_cast<uintptr_t>(1023));
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  // A kernel launched behind this one with a programmatic dependency (the
+  // recurrent step's fold of evicted keys) may be scheduled once every CTA
+  // has started: it reads nothing this kernel writes.
+  grid_dep_launch();
 
   // ---- unit -> (bh, chunk t, pair of 128-row query tiles) -----------------
   // Chunks are visited 1, 2, ..., n-1, 0: chunk 0 has no overlap frames (the
@@ -151,6 +156,7 @@ __global__ void __launch_bounds__(384, 1) hybrid_chunk_attn_kernel(const __grid_
       mbar_init(BAR(C::B_O + x), 1);
       mbar_init(BAR(C::B_PHI + x), 4);
       mbar_init(BAR(C::B_LIN + x), 1);
+      mbar_init(BAR(C::B_PVD + x), 1);
     }
     mbar_init(BAR(C::B_FIN), 1);
     *abort = 0;
@@ -451,6 +457,9 @@ __global__ void __launch_bounds__(384, 1) hybrid_chunk_attn_kernel(const __grid_
         load_tile(&p.tm_v, lo + 128 * j, -1);
       }
       if (has_lin) {
+        // The bf16 hi/lo state tiles come from the kernel before this one
+        // (launched with a programmatic dependency in the recurrent step).
+        grid_dep_wait();
         const int zc = bh * p.state_mul + (p.g.step ? 0 : t);
         for (int part = 0; part < 2 && ok; ++part)
           for (int rr = 0; rr < C::SPP && ok; ++rr) load_tile(part ? &p.tm_lo : &p.tm_hi, 128 * rr, zc);
@@ -522,9 +531,15 @@ __global__ void __launch_bounds__(384, 1) hybrid_chunk_attn_kernel(const __grid_
         const bool more = j + 1 < ntiles;
         ok = mbar_wait(BAR(C::B_FULL + vq % NS), (vq / NS) & 1, abort) && issue_PV(0, slot_addr(vq), j);
         if (!ok) break;
+        mma_commit(BAR(C::B_PVD + 0));
         TRACE(15, j);
         if (more) {
-          ok = mbar_wait(BAR(C::B_FULL + kn % NS), (kn / NS) & 1, abort);
+          // S_A(j+1) = Q_A K_{j+1}^T overwrites the TMEM columns P_A(j) occupies,
+          // the A operand of P_A(j) V_j: it is issued only once that MMA has
+          // completed (its commit), as tcgen05 operands must not be modified
+          // while an MMA that reads them is in flight.
+          ok = mbar_wait(BAR(C::B_FULL + kn % NS), (kn / NS) & 1, abort) &&
+               mbar_wait(BAR(C::B_PVD + 0), j & 1, abort);
           if (!ok) break;
           TRACE(14, j + 2);
           tc_fence_after();
@@ -538,7 +553,11 @@ __global__ void __launch_bounds__(384, 1) hybrid_chunk_attn_kernel(const __grid_
           ok = issue_PV(1, slot_addr(vq), j);
           if (!ok) break;
           mma_commit(BAR(C::B_EMPTY + vq % NS));
+          mma_commit(BAR(C::B_PVD + 1));
           if (more) {
+            ok = mbar_wait(BAR(C::B_PVD + 1), j & 1, abort);  // P_B(j) V_j complete (see S_A)
+            if (!ok) break;
+            tc_fence_after();
             issue_S(tmem + 128, lo_qB, slot_addr(kn));
             mma_commit(BAR(C::B_S + 1));
             TRACE(13, j);
@@ -594,26 +613,27 @@ __global__ void __launch_bounds__(384, 1) hybrid_chunk_attn_kernel(const __grid_
 int attn_smem_bytes(int D) { return D == 128 ? AttnCfg<128>::SMEM : AttnCfg<64>::SMEM; }
 
 template <int D, bool PARTS, bool PHI = false>
-static cudaError_t launch_attn_t(const AttnParams& p, int n_units, cudaStream_t s) {
+static cudaError_t launch_attn_t(const AttnParams& p, int n_units, cudaStream_t s, bool pdl) {
   auto* k = hybrid_chunk_attn_kernel<D, PARTS, PHI>;
   // The in-kernel register split assumes exactly REGS_LAUNCH registers per
   // thread at launch; with fewer, a warpgroup's increase could never be met.
   cudaError_t e = prepare_kernel_once(reinterpret_cast<const void*>(k), AttnCfg<D>::SMEM,
                                       static_cast<int>(AttnCfg<D>::REGS_LAUNCH));
   if (e != cudaSuccess) return e;
-  k<<<n_units, AttnCfg<D>::THREADS, AttnCfg<D>::SMEM, s>>>(p);
-  return cudaGetLastError();
+  return launch_k(k, dim3(n_units), dim3(AttnCfg<D>::THREADS), AttnCfg<D>::SMEM, s, pdl, p);
 }
 
-cudaError_t launch_attention(int D, bool parts, const AttnParams& p, int n_units, cudaStream_t s) {
+cudaError_t launch_attention(int D, bool parts, const AttnParams& p, int n_units, cudaStream_t s, bool pdl) {
   if (n_units <= 0) return cudaSuccess;
-  if (D == 128) return parts ? launch_attn_t<128, true>(p, n_units, s) : launch_attn_t<128, false>(p, n_units, s);
-  return parts ? launch_attn_t<64, true>(p, n_units, s) : launch_attn_t<64, false>(p, n_units, s);
+  if (D == 128)
+    return parts ? launch_attn_t<128, true>(p, n_units, s, pdl) : launch_attn_t<128, false>(p, n_units, s, pdl);
+  return parts ? launch_attn_t<64, true>(p, n_units, s, pdl) : launch_attn_t<64, false>(p, n_units, s, pdl);
 }
 
-cudaError_t launch_attention_phi(int D, const AttnParams& p, int n_units, cudaStream_t s) {
+cudaError_t launch_attention_phi(int D, const AttnParams& p, int n_units, cudaStream_t s, bool pdl) {
   if (n_units <= 0) return cudaSuccess;
-  return D == 128 ? launch_attn_t<128, false, true>(p, n_units, s) : launch_attn_t<64, false, true>(p, n_units, s);
+  return D == 128 ? launch_attn_t<128, false, true>(p, n_units, s, pdl)
+                  : launch_attn_t<64, false, true>(p, n_units, s, pdl);
 }
 
 }  // namespace rehyat
