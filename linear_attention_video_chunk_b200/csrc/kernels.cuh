@@ -40,6 +40,16 @@ struct AttnParams {
   float* Mo;
   const __nv_bfloat16* phi_q;  // [BH, N_q, 2D] precomputed phi(q) (feature-map variant only)
   unsigned long long* trace;   // clock64 stamps, only with -DREHYAT_TRACE (else unused)
+  // Units are numbered o = pair * BH + bh when pair_major (one chunk, the
+  // recurrent step), else o = (chunk order * BH + bh) * pairs + pair.  The
+  // n_split units o in [split_begin, split_begin + n_split) run as two CTAs
+  // each, over the first and the second half of the key window, and write
+  // partial rows instead of the output: launch index u runs o = u below
+  // split_begin, then the two halves of each split unit, then o = u - n_split.
+  int pair_major;
+  int split_begin;
+  int n_split;
+  float* part;        // [n_split, 2 halves, 2 query tiles, 128 rows, D + 4] fp32: O, denominator, shift, 2 pad
 };
 
 // phi(K)^T V and sum phi(K) over key segments (tensor cores).  One CTA =
@@ -143,6 +153,11 @@ cudaError_t launch_state_scan_bidir(const float* part_S, const float* part_z, in
                                     int n_chunks, int D, int Tc, int To, __nv_bfloat16* hi, __nv_bfloat16* lo,
                                     float* Sf, float* zt, cudaStream_t s);
 // state_S/z += sum over pieces of one segment's partials.
+// Combine the two key-window halves of every split unit (AttnParams): out =
+// (O0 2^(m0-M) + O1 2^(m1-M)) / (L0 2^(m0-M) + L1 2^(m1-M)), M = max(m0, m1).
+cudaError_t launch_split_merge(const float* part, int n_split, int split_begin, int BH, int H, int N_q, int D,
+                               __nv_bfloat16* out, long long o_sb, long long o_sh, long long o_sr, cudaStream_t s,
+                               bool pdl);
 cudaError_t launch_state_accumulate(const float* part_S, const float* part_z, int BH, int nsplit,
                                     int D, float* state_S, float* state_z, cudaStream_t s, bool pdl = false);
 // fp32 state -> bf16 hi/lo pair.

@@ -159,7 +159,8 @@ int apply_layout(int layout, FwdPlan* p) {
 struct StepPlan {
   int B, H;
   int BH, D, Nq, Nk, evict_tok, nsplit, pairs, n_units;
-  size_t off_hi, off_lo, off_pS, off_pz, bytes;
+  int split_begin, n_split;  // key-window split of the attention's last wave (AttnParams)
+  size_t off_hi, off_lo, off_pS, off_pz, off_part, bytes;
   size_t f32_off_pS, f32_off_pz, f32_bytes;
 };
 
@@ -187,12 +188,30 @@ int plan_step(int B, int H, int S_tok, int d, int qf, int cf, int ef, StepPlan* 
   const long long units = BH * p->pairs;
   if (units > INT_MAX) return REHYAT_EINVAL;
   p->n_units = static_cast<int>(units);
+  // The attention's units are ordered pair-major, so the units with a
+  // single query tile (the ragged last pair) come last.  When the units do
+  // not fill a whole number of waves of kSplitTarget CTAs, the last full
+  // units run as two CTAs over the two halves of the key window, as many as
+  // fit beside the single-tile units in one last wave (needs >= 2 key tiles).
+  {
+    const int U = p->n_units;
+    const int U_t = (cdiv(p->Nq, 128) % 2) ? p->BH : 0;
+    const int R = U % kSplitTarget;
+    int s_ = 0;
+    if (U > kSplitTarget && R > 0 && cdiv(p->Nk, 128) >= 2) {
+      s_ = imin(R - U_t, kSplitTarget - R);
+      if (s_ < 0) s_ = 0;
+    }
+    p->n_split = s_;
+    p->split_begin = (U - U_t) - s_;
+  }
   const size_t D2 = 2 * static_cast<size_t>(d);
   size_t off = 0;
   p->off_hi = off; off += align256(static_cast<size_t>(BH) * D2 * d * 2);
   p->off_lo = off; off += align256(static_cast<size_t>(BH) * D2 * d * 2);
   p->off_pS = off; off += align256(static_cast<size_t>(BH) * p->nsplit * D2 * d * 4);
   p->off_pz = off; off += align256(static_cast<size_t>(BH) * p->nsplit * D2 * 4);
+  p->off_part = off; off += align256(static_cast<size_t>(p->n_split) * 2 * 2 * 128 * (d + 4) * 4);
   p->bytes = off;
   off = 0;
   p->f32_off_pS = off; off += align256(static_cast<size_t>(BH) * D2 * d * 4);
@@ -847,6 +866,10 @@ int run_step(const void* q_c, const void* k_c, const void* v_c, const void* phi_
   ap.o_sh = q_hs;
   ap.o_sr = q_rs;
   ap.pairs = P.pairs;
+  ap.pair_major = 1;
+  ap.split_begin = P.split_begin;
+  ap.n_split = P.n_split;
+  ap.part = reinterpret_cast<float*>(w + P.off_part);
   ap.state_mul = 1;
   ap.scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(P.D));
   ap.z = state_z;
@@ -859,12 +882,16 @@ int run_step(const void* q_c, const void* k_c, const void* v_c, const void* phi_
   // attention's last wave leaves idle; each kernel waits before it touches
   // what an earlier one writes (the attention before its state tiles, the
   // update before everything).
+  const int n_ctas = P.n_units + P.n_split;
   if (phi_q != nullptr) {
     ap.phi_q = static_cast<const __nv_bfloat16*>(phi_q);
-    st = cuda_status(launch_attention_phi(P.D, ap, P.n_units, s, true));
+    st = cuda_status(launch_attention_phi(P.D, ap, n_ctas, s, true));
   } else {
-    st = cuda_status(launch_attention(P.D, false, ap, P.n_units, s, true));
+    st = cuda_status(launch_attention(P.D, false, ap, n_ctas, s, true));
   }
+  if (st == REHYAT_OK)
+    st = cuda_status(launch_split_merge(ap.part, P.n_split, P.split_begin, P.BH, P.H, P.Nq, P.D, ap.out, ap.o_sb,
+                                        ap.o_sh, ap.o_sr, s, true));
   if (st != REHYAT_OK || P.evict_tok == 0) return st;
   StateParams sp;
   std::memset(&sp, 0, sizeof(sp));

@@ -137,6 +137,51 @@ int grid_for(long long n, int threads) {
   return static_cast<int>(g < 1 ? 1 : g);
 }
 
+// The two key-window halves of every split unit of the fused attention:
+// one thread per (split unit, query tile, row, group of 8 columns).  The
+// partial rows hold O (unnormalised, scaled by 2^-m), the denominator L on
+// the same scale, and the shift m (log2 units); the halves combine on the
+// larger shift.  Launched with a programmatic dependency right behind the
+// attention, so it waits for it first.
+__global__ void split_merge_kernel(const float* __restrict__ part, int n_split, int split_begin, int BH, int H,
+                                   int N_q, int D, __nv_bfloat16* __restrict__ out, long long o_sb, long long o_sh,
+                                   long long o_sr) {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  const int G8 = D / 8;
+  const long long total = static_cast<long long>(n_split) * 2 * 128 * G8;
+  const size_t W = static_cast<size_t>(D) + 4;
+  for (long long idx = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; idx < total;
+       idx += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const int g = static_cast<int>(idx % G8);
+    const long long rr = idx / G8;
+    const int r = static_cast<int>(rr % 128);
+    const int X = static_cast<int>((rr / 128) % 2);
+    const int i = static_cast<int>(rr / 256);
+    const int o = split_begin + i;  // pair-major unit number
+    const int pair = o / BH, bh = o % BH;
+    const int qrow = pair * 256 + X * 128 + r;
+    if (qrow >= N_q) continue;
+    const float* e0 = part + ((static_cast<size_t>(i * 2 + 0) * 2 + X) * 128 + r) * W;
+    const float* e1 = part + ((static_cast<size_t>(i * 2 + 1) * 2 + X) * 128 + r) * W;
+    const float m0 = e0[D + 1], m1 = e1[D + 1];
+    const float M = fmaxf(m0, m1);
+    const float w0 = exp2f(m0 - M), w1 = exp2f(m1 - M);
+    const float inv = 1.f / (e0[D] * w0 + e1[D] * w1);
+    const float4 a0 = reinterpret_cast<const float4*>(e0 + 8 * g)[0], b0 = reinterpret_cast<const float4*>(e0 + 8 * g)[1];
+    const float4 a1 = reinterpret_cast<const float4*>(e1 + 8 * g)[0], b1 = reinterpret_cast<const float4*>(e1 + 8 * g)[1];
+    const float y[8] = {a0.x * w0 + a1.x * w1, a0.y * w0 + a1.y * w1, a0.z * w0 + a1.z * w1, a0.w * w0 + a1.w * w1,
+                        b0.x * w0 + b1.x * w1, b0.y * w0 + b1.y * w1, b0.z * w0 + b1.z * w1, b0.w * w0 + b1.w * w1};
+    uint32_t pk[4];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      __nv_bfloat162 h2 = __floats2bfloat162_rn(y[2 * c] * inv, y[2 * c + 1] * inv);
+      pk[c] = *reinterpret_cast<uint32_t*>(&h2);
+    }
+    *reinterpret_cast<uint4*>(out + (bh / H) * o_sb + (bh % H) * o_sh + qrow * o_sr + 8 * g) =
+        make_uint4(pk[0], pk[1], pk[2], pk[3]);
+  }
+}
+
 }  // namespace
 
 cudaError_t launch_state_scan(const float* part_S, const float* part_z, int BH, int n_seg, int nsplit,
@@ -162,6 +207,15 @@ cudaError_t launch_state_accumulate(const float* part_S, const float* part_z, in
   const long long n = static_cast<long long>(BH) * 2 * D * (D + 1);
   return launch_k(state_accumulate_kernel, dim3(grid_for(n, 256)), dim3(256), 0, s, pdl, part_S, part_z, BH, nsplit,
                   D, state_S, state_z);
+}
+
+cudaError_t launch_split_merge(const float* part, int n_split, int split_begin, int BH, int H, int N_q, int D,
+                               __nv_bfloat16* out, long long o_sb, long long o_sh, long long o_sr, cudaStream_t s,
+                               bool pdl) {
+  if (n_split <= 0) return cudaSuccess;
+  const long long n = static_cast<long long>(n_split) * 2 * 128 * (D / 8);
+  return launch_k(split_merge_kernel, dim3(grid_for(n, 256)), dim3(256), 0, s, pdl, part, n_split, split_begin, BH,
+                  H, N_q, D, out, o_sb, o_sh, o_sr);
 }
 
 cudaError_t launch_state_split(const float* S, long long n, __nv_bfloat16* hi, __nv_bfloat16* lo,

@@ -118,15 +118,40 @@ __global__ void __launch_bounds__(384, 1) hybrid_chunk_attn_kernel(const __grid_
 
   // ---- unit -> (bh, chunk t, pair of 128-row query tiles) -----------------
   // Chunks are visited 1, 2, ..., n-1, 0: chunk 0 has no overlap frames (the
-  // shortest window), so the longest units start first.
+  // shortest window), so the longest units start first.  A split unit's two
+  // CTAs (half 0 and 1) each take half of the key window's tiles.
   const int u = blockIdx.x;
-  const int pair = u % p.pairs;
-  const int rest = u / p.pairs;
-  const int bh = rest % p.BH;
-  const int o = rest / p.BH;
-  const int t = (p.g.n_chunks > 1) ? (o + 1) % p.g.n_chunks : 0;
+  int ou = u, half = -1;
+  if (p.n_split > 0 && u >= p.split_begin) {
+    const int v = u - p.split_begin;
+    if (v < 2 * p.n_split) {
+      ou = p.split_begin + (v >> 1);
+      half = v & 1;
+    } else {
+      ou = u - p.n_split;
+    }
+  }
+  int pair, bh, t;
+  if (p.pair_major) {
+    pair = ou / p.BH;
+    bh = ou % p.BH;
+    t = 0;
+  } else {
+    pair = ou % p.pairs;
+    const int rest = ou / p.pairs;
+    bh = rest % p.BH;
+    const int o = rest / p.BH;
+    t = (p.g.n_chunks > 1) ? (o + 1) % p.g.n_chunks : 0;
+  }
   int q0, q1, lo, hi;
   p.g.chunk(t, q0, q1, lo, hi);
+  if (half >= 0) {
+    const int h0 = (cdiv(hi - lo, 128) + 1) / 2;  // tiles of the first half
+    if (half == 0)
+      hi = lo + 128 * h0;
+    else
+      lo += 128 * h0;
+  }
   const int rowA0 = q0 + pair * 256;
   const int rowB0 = rowA0 + 128;
   const int nA = imin(imax(q1 - rowA0, 0), 128);
@@ -165,7 +190,7 @@ __global__ void __launch_bounds__(384, 1) hybrid_chunk_attn_kernel(const __grid_
   if (warp == 1) {
     // The linear set is non-empty iff z_t > 0 somewhere (phi > 0 elementwise).
     int f = 0;
-    if (p.z != nullptr) {
+    if (p.z != nullptr && half != 1) {  // the linear term is added by the first half of a split unit
       const float* zp = p.z + bh * p.z_bh + t * p.z_t;
       for (int e = lane; e < 2 * D; e += 32) f |= (zp[e] > 0.f) ? 1 : 0;
     }
@@ -377,7 +402,25 @@ __global__ void __launch_bounds__(384, 1) hybrid_chunk_attn_kernel(const __grid_
         tc_fence_after();
       }
 
-      if (ok) {
+      if (ok && !PARTS && half >= 0) {
+        // split unit: the partial row (unnormalised O, its denominator and
+        // shift, log2 units) for the merge
+        float* e = p.part + ((static_cast<size_t>((ou - p.split_begin) * 2 + half) * 2 + X) * 128 + r) * (D + 4);
+#pragma unroll
+        for (int a = 0; a < D / 32; ++a) {
+          uint32_t ov[32];
+          tmem_ld32(tO + 32 * a, ov);
+          tmem_ld_wait();
+          reg_fence(ov);
+          float4* dst = reinterpret_cast<float4*>(e + 32 * a);
+#pragma unroll
+          for (int c = 0; c < 8; ++c)
+            dst[c] = make_float4(__uint_as_float(ov[4 * c]), __uint_as_float(ov[4 * c + 1]),
+                                 __uint_as_float(ov[4 * c + 2]), __uint_as_float(ov[4 * c + 3]));
+        }
+        e[D] = l + nl;
+        e[D + 1] = m_used;
+      } else if (ok) {
         if (!PARTS) {
           const float inv = 1.f / (l + nl);
 #pragma unroll

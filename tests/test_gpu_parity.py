@@ -314,6 +314,29 @@ def test_step_from_nonzero_state_matches_oracle_step():
     assert np.abs(np64(zd) - oz).max() / np.abs(oz).max() < 1e-3
 
 
+@pytest.mark.parametrize("d", [128, 64])
+def test_step_last_wave_split_matches_oracle(d):
+    """B=1, H=20, 780 tokens a frame, 3 query frames after 1 overlap frame:
+    the fused attention has 200 units (20 with a single query tile) for 148
+    SMs, so the last 32 full units run as two CTAs over the halves of the key
+    window and are merged.  From a non-zero state (the first half carries the
+    linear term), every row of three heads against the oracle's step (every
+    head has split units, heads 8-19 two of them), bitwise repeatable."""
+    B, H, S, qf, cf, ef = 1, 20, 780, 3, 1, 1
+    q, _, _ = inputs.make_qkv(B, H, qf * S, d, 180, rms_qk=True)
+    _, k, v = inputs.make_qkv(B, H, (cf + qf) * S, d, 181, rms_qk=True)
+    S0, z0 = inputs.make_state(B, H, d, 182, scale=30.0)
+    qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+    Sd, zd = S0.cuda(), z0.cuda()
+    y = R.step(qd, kd, vd, Sd, zd, S, qf, cf, ef)
+    y2 = R.step(qd, kd, vd, S0.cuda(), z0.cuda(), S, qf, cf, ef)
+    assert torch.equal(y, y2)
+    yn = np64(y)
+    for h in (0, 8, 19):
+        oy, _, _ = orc.oracle_step(q[:, h:h + 1], k[:, h:h + 1], v[:, h:h + 1], S0[:, h:h + 1], z0[:, h:h + 1], S, ef)
+        assert_bf16_close(yn[:, h:h + 1], oy, f"head {h}")
+
+
 def test_deterministic_bitwise():
     B, H, d, F, S, Tc, To = 1, 3, 128, 7, 110, 3, 1
     q, k, v = (x.cuda() for x in inputs.make_qkv(B, H, F * S, d, 90, rms_qk=True))
