@@ -282,9 +282,11 @@ int rehyat_forward_parts(const void* q, const void* k, const void* v,
                          void* stream);
 
 /* States entering each chunk, exported for inspection (bf16 inputs,
- * tensor-core phi(K)^T V, fp32 scan):  S [B,H,n_chunks,2d,d] fp32,
- * z [B,H,n_chunks,2d] fp32 with n_chunks = ceil(F / chunk_frames);
- * S_t = sum_{j < lo_t} phi(k_j) v_j^T, z_t = sum_{j < lo_t} phi(k_j). */
+ * tensor-core phi(K)^T V, fp32 scan):  S [B,H,n_chunks,2d,d] fp32 (device,
+ * caller-owned, 16-byte aligned), z [B,H,n_chunks,2d] fp32 (device,
+ * caller-owned) with n_chunks = ceil(F / chunk_frames);
+ * S_t = sum_{j < lo_t} phi(k_j) v_j^T, z_t = sum_{j < lo_t} phi(k_j).
+ * Returns REHYAT_EINVAL for null or misaligned pointers or bad sizes. */
 int rehyat_chunk_states(const void* k, const void* v,
                         int B, int H, int F, int S_tok, int d,
                         int chunk_frames, int overlap_frames,

@@ -737,7 +737,7 @@ REHYAT_API int rehyat_chunk_states(const void* k, const void* v, int B, int H, i
   FwdPlan P;
   int st = plan_forward(B, H, F, S_tok, d, chunk_frames, overlap_frames, &P);
   if (st != REHYAT_OK) return st;
-  if (check_ptr(k) || check_ptr(v) || S == nullptr || z == nullptr) return REHYAT_EINVAL;
+  if (check_ptr(k) || check_ptr(v) || check_ptr(S) || z == nullptr) return REHYAT_EINVAL;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   WsGuard ws(s);
   st = ws.alloc(P.off_hi);  // partials only

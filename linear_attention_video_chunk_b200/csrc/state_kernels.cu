@@ -16,107 +16,167 @@ namespace {
 // ============================================================================
 // Scan / accumulate / split (SIMT, memory-bound)
 // ============================================================================
-// One thread per state entry (bh, e, c) with c == D meaning z: walks the
-// chunks in order, writing the exclusive prefix, then adding segment t.
+// The vector kernels below give each thread four consecutive state columns
+// (one float4) of one row e of one (b,h); the thread holding columns 0..3
+// also carries z[e].  Every pointer is 16-byte aligned and D % 4 == 0, so
+// the float4 loads and 8-byte bf16 stores are aligned.
+struct Row4 {
+  int bh, e, c;  // c = first of the four columns
+  bool z;        // this thread also carries z[e]
+};
+__device__ __forceinline__ Row4 row4(long long idx, int D) {
+  // D is 64 or 128: D / 4 and 2D are powers of two (shifts, no division)
+  const int lg = (D == 128) ? 5 : 4;  // log2(D / 4); log2(2D) = lg + 3
+  Row4 r;
+  r.c = 4 * static_cast<int>(idx & ((1 << lg) - 1));
+  r.e = static_cast<int>((idx >> lg) & ((2 * D) - 1));
+  r.bh = static_cast<int>(idx >> (2 * lg + 3));
+  r.z = r.c == 0;
+  return r;
+}
+__device__ __forceinline__ void add4(float4& a, const float4 b) {
+  a.x += b.x;
+  a.y += b.y;
+  a.z += b.z;
+  a.w += b.w;
+}
+// The state entering a chunk: fp32 (Sf) or the bf16 pair hi = bf16(S),
+// lo = bf16(S - hi) the tensor-core epilogue reads.
+__device__ __forceinline__ void put_state(size_t so, const Row4& r, int D, const float4 acc, float az,
+                                          __nv_bfloat16* __restrict__ hi, __nv_bfloat16* __restrict__ lo,
+                                          float* __restrict__ Sf, float* __restrict__ zt) {
+  if (r.z) zt[so] = az;
+  const size_t o = so * D + r.c;
+  if (hi != nullptr) {
+    const float v[4] = {acc.x, acc.y, acc.z, acc.w};
+    __nv_bfloat16 h[4], l[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      h[i] = __float2bfloat16_rn(v[i]);
+      l[i] = __float2bfloat16_rn(v[i] - __bfloat162float(h[i]));
+    }
+    *reinterpret_cast<uint2*>(hi + o) = *reinterpret_cast<const uint2*>(h);
+    *reinterpret_cast<uint2*>(lo + o) = *reinterpret_cast<const uint2*>(l);
+  } else {
+    *reinterpret_cast<float4*>(Sf + o) = acc;
+  }
+}
+
+// Exclusive scan over chunks: chunk t receives the sum of segments 0..t-1,
+// each segment the sum of its pieces in piece order.  The (segment, piece)
+// items are read eight at a time ahead of the sums (the loads do not depend
+// on them; past the last item the index is clamped, so every load is valid).
 __global__ void state_scan_kernel(const float* __restrict__ pS, const float* __restrict__ pz, int BH,
-                                  int n_seg, int nsplit, int nc, int D, __nv_bfloat16* hi,
-                                  __nv_bfloat16* lo, float* Sf, float* zt) {
-  const int W = D + 1;
-  const long long total = static_cast<long long>(BH) * 2 * D * W;
+                                  int n_seg, int nsplit, int nc, int D, __nv_bfloat16* __restrict__ hi,
+                                  __nv_bfloat16* __restrict__ lo, float* __restrict__ Sf, float* __restrict__ zt) {
+  constexpr int PF = 8;
+  const long long total = static_cast<long long>(BH) * 2 * D * (D / 4);
+  const int n_items = n_seg * nsplit;  // per (b,h); the planner bounds BH * n_items by INT_MAX
   for (long long idx = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; idx < total;
        idx += static_cast<long long>(gridDim.x) * blockDim.x) {
-    const int c = static_cast<int>(idx % W);
-    const int e = static_cast<int>((idx / W) % (2 * D));
-    const int bh = static_cast<int>(idx / (static_cast<long long>(W) * 2 * D));
-    float acc = 0.f;
-    for (int t = 0; t < nc; ++t) {
-      const size_t so = ((static_cast<size_t>(bh) * nc + t) * 2 * D + e);
-      if (c == D) {
-        zt[so] = acc;
-      } else if (hi != nullptr) {
-        const __nv_bfloat16 h = __float2bfloat16_rn(acc);
-        hi[so * D + c] = h;
-        lo[so * D + c] = __float2bfloat16_rn(acc - __bfloat162float(h));
-      } else {
-        Sf[so * D + c] = acc;
+    const Row4 r = row4(idx, D);
+    const size_t so0 = static_cast<size_t>(r.bh) * nc * 2 * D + r.e;  // (bh, t = 0, e)
+    const size_t po0 = static_cast<size_t>(r.bh) * n_items;           // (bh, segment 0, piece 0)
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    float az = 0.f;
+    int t_next = 0;  // the next chunk whose state is still to be written
+    int pp = 0;      // piece of the next item
+    for (int j0 = 0; j0 < n_items; j0 += PF) {
+      float4 v[PF];
+      float vz[PF];
+#pragma unroll
+      for (int i = 0; i < PF; ++i) {
+        const size_t po = po0 + static_cast<size_t>(imin(j0 + i, n_items - 1));
+        v[i] = __ldg(reinterpret_cast<const float4*>(pS + (po * 2 * D + r.e) * D + r.c));
+        vz[i] = r.z ? __ldg(pz + po * 2 * D + r.e) : 0.f;
       }
-      if (t < n_seg) {
-        for (int pp = 0; pp < nsplit; ++pp) {
-          const size_t po = (static_cast<size_t>(bh) * n_seg + t) * nsplit + pp;
-          acc += (c == D) ? pz[po * 2 * D + e] : pS[(po * 2 * D + e) * D + c];
+#pragma unroll
+      for (int i = 0; i < PF; ++i) {
+        if (j0 + i < n_items) {
+          if (pp == 0)  // the first piece of segment t_next: chunk t_next's prefix is complete
+            put_state(so0 + static_cast<size_t>(t_next++) * 2 * D, r, D, acc, az, hi, lo, Sf, zt);
+          add4(acc, v[i]);
+          az += vz[i];
+          if (++pp == nsplit) pp = 0;
         }
       }
     }
+    for (; t_next < nc; ++t_next) put_state(so0 + static_cast<size_t>(t_next) * 2 * D, r, D, acc, az, hi, lo, Sf, zt);
   }
 }
 
 // Bidirectional sets: segments are frames; for chunk t with window frames
 // [lo_f, hi_f) the state is sum over frames < lo_f plus frames >= hi_f.  One
-// thread per state entry walks the frames twice (total, then the two
+// thread per four state entries walks the frames twice (total, then the two
 // monotone prefix pointers), in a fixed order.
 __global__ void state_scan_bidir_kernel(const float* __restrict__ pS, const float* __restrict__ pz, int BH,
-                                        int F, int nsplit, int nc, int D, int Tc, int To, __nv_bfloat16* hi,
-                                        __nv_bfloat16* lo, float* Sf, float* zt) {
-  const int W = D + 1;
-  const long long total = static_cast<long long>(BH) * 2 * D * W;
+                                        int F, int nsplit, int nc, int D, int Tc, int To,
+                                        __nv_bfloat16* __restrict__ hi, __nv_bfloat16* __restrict__ lo,
+                                        float* __restrict__ Sf, float* __restrict__ zt) {
+  const long long total = static_cast<long long>(BH) * 2 * D * (D / 4);
   for (long long idx = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; idx < total;
        idx += static_cast<long long>(gridDim.x) * blockDim.x) {
-    const int c = static_cast<int>(idx % W);
-    const int e = static_cast<int>((idx / W) % (2 * D));
-    const int bh = static_cast<int>(idx / (static_cast<long long>(W) * 2 * D));
-    auto frame = [&](int f) {
-      float acc = 0.f;
+    const Row4 r = row4(idx, D);
+    auto frame = [&](int f, float& fz) {
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      fz = 0.f;
       for (int pp = 0; pp < nsplit; ++pp) {
-        const size_t po = (static_cast<size_t>(bh) * F + f) * nsplit + pp;
-        acc += (c == D) ? pz[po * 2 * D + e] : pS[(po * 2 * D + e) * D + c];
+        const size_t po = (static_cast<size_t>(r.bh) * F + f) * nsplit + pp;
+        add4(acc, __ldg(reinterpret_cast<const float4*>(pS + (po * 2 * D + r.e) * D + r.c)));
+        if (r.z) fz += __ldg(pz + po * 2 * D + r.e);
       }
       return acc;
     };
-    float tot = 0.f;
-    for (int f = 0; f < F; ++f) tot += frame(f);
-    float p_lo = 0.f, p_hi = 0.f;  // prefix sums up to lo_f and hi_f
+    float4 tot = make_float4(0.f, 0.f, 0.f, 0.f);
+    float tz = 0.f, fz;
+    for (int f = 0; f < F; ++f) {
+      add4(tot, frame(f, fz));
+      tz += fz;
+    }
+    float4 p_lo = make_float4(0.f, 0.f, 0.f, 0.f), p_hi = p_lo;  // prefix sums up to lo_f and hi_f
+    float z_lo = 0.f, z_hi = 0.f;
     int f_lo = 0, f_hi = 0;
     for (int t = 0; t < nc; ++t) {
       const int lo_f = imax(t * Tc - To, 0), hi_f = imin((t + 1) * Tc, F);
-      for (; f_lo < lo_f; ++f_lo) p_lo += frame(f_lo);
-      for (; f_hi < hi_f; ++f_hi) p_hi += frame(f_hi);
-      const float acc = p_lo + (tot - p_hi);
-      const size_t so = ((static_cast<size_t>(bh) * nc + t) * 2 * D + e);
-      if (c == D) {
-        zt[so] = acc;
-      } else if (hi != nullptr) {
-        const __nv_bfloat16 h = __float2bfloat16_rn(acc);
-        hi[so * D + c] = h;
-        lo[so * D + c] = __float2bfloat16_rn(acc - __bfloat162float(h));
-      } else {
-        Sf[so * D + c] = acc;
+      for (; f_lo < lo_f; ++f_lo) {
+        add4(p_lo, frame(f_lo, fz));
+        z_lo += fz;
       }
+      for (; f_hi < hi_f; ++f_hi) {
+        add4(p_hi, frame(f_hi, fz));
+        z_hi += fz;
+      }
+      const float4 acc = make_float4(p_lo.x + (tot.x - p_hi.x), p_lo.y + (tot.y - p_hi.y), p_lo.z + (tot.z - p_hi.z),
+                                     p_lo.w + (tot.w - p_hi.w));
+      put_state(static_cast<size_t>(r.bh) * nc * 2 * D + static_cast<size_t>(t) * 2 * D + r.e, r, D, acc,
+                z_lo + (tz - z_hi), hi, lo, Sf, zt);
     }
   }
 }
 
 __global__ void state_accumulate_kernel(const float* __restrict__ pS, const float* __restrict__ pz, int BH,
-                                        int nsplit, int D, float* S, float* z) {
+                                        int nsplit, int D, float* __restrict__ S, float* __restrict__ z) {
   // In the recurrent step this kernel follows the fold of evicted keys with
   // a programmatic dependency: wait until that fold (and so the attention
   // before it, which reads z) has completed.
   asm volatile("griddepcontrol.wait;" ::: "memory");
-  const int W = D + 1;
-  const long long total = static_cast<long long>(BH) * 2 * D * W;
+  const long long total = static_cast<long long>(BH) * 2 * D * (D / 4);
   for (long long idx = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; idx < total;
        idx += static_cast<long long>(gridDim.x) * blockDim.x) {
-    const int c = static_cast<int>(idx % W);
-    const int e = static_cast<int>((idx / W) % (2 * D));
-    const int bh = static_cast<int>(idx / (static_cast<long long>(W) * 2 * D));
-    float acc = 0.f;
+    const Row4 r = row4(idx, D);
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    float az = 0.f;
     for (int pp = 0; pp < nsplit; ++pp) {
-      const size_t po = static_cast<size_t>(bh) * nsplit + pp;
-      acc += (c == D) ? pz[po * 2 * D + e] : pS[(po * 2 * D + e) * D + c];
+      const size_t po = static_cast<size_t>(r.bh) * nsplit + pp;
+      add4(acc, __ldg(reinterpret_cast<const float4*>(pS + (po * 2 * D + r.e) * D + r.c)));
+      if (r.z) az += __ldg(pz + po * 2 * D + r.e);
     }
-    if (c == D)
-      z[static_cast<size_t>(bh) * 2 * D + e] += acc;
-    else
-      S[(static_cast<size_t>(bh) * 2 * D + e) * D + c] += acc;
+    const size_t so = static_cast<size_t>(r.bh) * 2 * D + r.e;
+    float4* dst = reinterpret_cast<float4*>(S + so * D + r.c);
+    float4 cur = *dst;
+    add4(cur, acc);
+    *dst = cur;
+    if (r.z) z[so] += az;
   }
 }
 
@@ -187,7 +247,7 @@ __global__ void split_merge_kernel(const float* __restrict__ part, int n_split, 
 cudaError_t launch_state_scan(const float* part_S, const float* part_z, int BH, int n_seg, int nsplit,
                               int n_chunks, int D, __nv_bfloat16* hi, __nv_bfloat16* lo, float* Sf,
                               float* zt, cudaStream_t s) {
-  const long long n = static_cast<long long>(BH) * 2 * D * (D + 1);
+  const long long n = static_cast<long long>(BH) * 2 * D * (D / 4);
   state_scan_kernel<<<grid_for(n, 256), 256, 0, s>>>(part_S, part_z, BH, n_seg, nsplit, n_chunks, D, hi, lo,
                                                       Sf, zt);
   return cudaGetLastError();
@@ -196,7 +256,7 @@ cudaError_t launch_state_scan(const float* part_S, const float* part_z, int BH, 
 cudaError_t launch_state_scan_bidir(const float* part_S, const float* part_z, int BH, int F, int nsplit,
                                     int n_chunks, int D, int Tc, int To, __nv_bfloat16* hi, __nv_bfloat16* lo,
                                     float* Sf, float* zt, cudaStream_t s) {
-  const long long n = static_cast<long long>(BH) * 2 * D * (D + 1);
+  const long long n = static_cast<long long>(BH) * 2 * D * (D / 4);
   state_scan_bidir_kernel<<<grid_for(n, 256), 256, 0, s>>>(part_S, part_z, BH, F, nsplit, n_chunks, D, Tc, To, hi,
                                                             lo, Sf, zt);
   return cudaGetLastError();
@@ -204,7 +264,7 @@ cudaError_t launch_state_scan_bidir(const float* part_S, const float* part_z, in
 
 cudaError_t launch_state_accumulate(const float* part_S, const float* part_z, int BH, int nsplit, int D,
                                     float* state_S, float* state_z, cudaStream_t s, bool pdl) {
-  const long long n = static_cast<long long>(BH) * 2 * D * (D + 1);
+  const long long n = static_cast<long long>(BH) * 2 * D * (D / 4);
   return launch_k(state_accumulate_kernel, dim3(grid_for(n, 256)), dim3(256), 0, s, pdl, part_S, part_z, BH, nsplit,
                   D, state_S, state_z);
 }

@@ -84,6 +84,15 @@ def test_step_validation(lib):
     assert st(d=32) == R.EUNSUPPORTED
 
 
+def test_chunk_states_validation(lib):
+    # k, v, S: 16-byte aligned device pointers; z: non-null
+    f = lib.rehyat_chunk_states
+    assert f(16, 16, 1, 1, 4, 8, 64, 2, 1, 0, 16, None) == R.EINVAL    # null S
+    assert f(16, 16, 1, 1, 4, 8, 64, 2, 1, 20, 16, None) == R.EINVAL   # S at 4 mod 16
+    assert f(16, 16, 1, 1, 4, 8, 64, 2, 1, 16, 0, None) == R.EINVAL    # null z
+    assert f(8, 16, 1, 1, 4, 8, 64, 2, 1, 16, 16, None) == R.EINVAL    # misaligned k
+
+
 def test_workspace_sizes(lib):
     a = R.workspace_bytes(1, 12, 21, 1560, 128, 3, 1)
     b = R.workspace_bytes(1, 12, 41, 1560, 128, 3, 1)
