@@ -25,8 +25,9 @@ namespace {
 //   phi = [1 + elu(U_1 + b2_1), (1 + elu(U_2 + b2_2))^2]   bf16 -> global
 // Warps 0-15 run both epilogues: warp w reads TMEM lane quarter w % 4 and
 // column group w / 4 (a quarter of H's and of U's columns); warp 16 is the TMA
-// producer, warp 17 the MMA issuer.  The next H GEMM runs while the epilogue
-// still reads U.  Features leave through shared memory and TMA tile stores
+// producer, warp 17 the MMA issuer.  The next H GEMM (issued once the second
+// GEMM, which reads R from H's columns, has completed) runs while the
+// epilogue still reads U.  Features leave through shared memory and TMA tile stores
 // (32 features x 128 rows a box, one box per group and chunk step), so each
 // row is written whole instead of 16 bytes per thread at a 2D-element
 // stride; the producer thread issues those stores and waits for them, so the
@@ -273,6 +274,10 @@ __global__ void __launch_bounds__(MlpCfg<D>::THREADS, 1) phi_mlp_kernel(const __
       for (int it = 0; it < my_tiles && ok; ++it) {
         const int slot = it % C::NXB;
         ok = mbar_wait(BAR(C::B_X + slot), (it / C::NXB) & 1, abort);
+        // H overwrites the TMEM columns that hold R of the previous tile, the
+        // A operand of its second GEMM: issued only once that GEMM has
+        // completed (tcgen05 operands must not change under an MMA in flight)
+        if (ok && it > 0) ok = mbar_wait(BAR(C::B_U), (it - 1) & 1, abort);
         if (!ok) break;
         TRACE(8, it);
         tc_fence_after();
