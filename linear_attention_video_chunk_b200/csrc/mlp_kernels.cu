@@ -62,14 +62,23 @@ struct MlpCfg {
   static constexpr uint32_t TMEM_COLS = (HID + OUT <= 256) ? 256u : 512u;
   static constexpr int EPI_WARPS = 4 * NG;
   static constexpr int THREADS = 32 * EPI_WARPS + 64;
+  // At D = 128 the second GEMM runs as two N = 128 halves of U (features
+  // [0, D) and [D, 2D)), each with its own ready / free barrier, so the
+  // features of the first half are computed while the tensor core produces
+  // the second.  Epilogue group g takes features 32g.. of each half (one
+  // 32-feature chunk a half).  At D = 64 a half would be 16 features a group,
+  // under a chunk: one N = 2D GEMM, group g takes features g * OG...
+  static constexpr bool SPLIT = (D == 128);
+  static constexpr int NU = SPLIT ? 2 : 1;          // U halves
   static constexpr int B_W = 0, B_X = 1, B_XE = 1 + NXB, B_H = 1 + 2 * NXB, B_R = B_H + 1, B_U = B_H + 2,
-                       B_UE = B_H + 3, B_STF = B_H + 4, B_STE = B_H + 5, B_FIN = B_H + 6;
+                       B_UE = B_U + 2, B_STF = B_UE + 2, B_STE = B_STF + 1, B_FIN = B_STE + 1;
   static constexpr int NC = OG / 32;                // 32-feature chunk steps of a tile
+  static_assert(!SPLIT || NC == NU, "one chunk per U half");
   static_assert(!ALIAS || (NXB == 1 && X_BYTES >= STG_STEP), "staging inside the x tile");
   static_assert(HG % 32 == 0 && OG % 32 == 0, "whole 32-column chunks per group");
   // both GEMMs: A and B K-major (x rows / R rows by W rows)
   static constexpr uint32_t IDESC1 = idesc_bf16_f32(128, HID, 0, 0);
-  static constexpr uint32_t IDESC2 = idesc_bf16_f32(128, OUT, 0, 0);
+  static constexpr uint32_t IDESC2 = idesc_bf16_f32(128, OUT / NU, 0, 0);
   static_assert(SMEM <= 232448, "shared memory");
   static_assert((B_FIN + 1) * 8 <= 128, "barrier area");
   static_assert(HID + OUT <= 512, "tensor memory");
@@ -105,8 +114,10 @@ __global__ void __launch_bounds__(MlpCfg<D>::THREADS, 1) phi_mlp_kernel(const __
     }
     mbar_init(BAR(C::B_H), 1);
     mbar_init(BAR(C::B_R), C::EPI_WARPS);
-    mbar_init(BAR(C::B_U), 1);
-    mbar_init(BAR(C::B_UE), C::EPI_WARPS);
+    for (int h = 0; h < 2; ++h) {
+      mbar_init(BAR(C::B_U + h), 1);
+      mbar_init(BAR(C::B_UE + h), C::EPI_WARPS);
+    }
     mbar_init(BAR(C::B_STF), C::EPI_WARPS);
     mbar_init(BAR(C::B_STE), 1);
     mbar_init(BAR(C::B_FIN), 1);
@@ -133,8 +144,6 @@ __global__ void __launch_bounds__(MlpCfg<D>::THREADS, 1) phi_mlp_kernel(const __
     const int quarter = warp & 3, g = warp >> 2;
     const uint32_t lane_off = static_cast<uint32_t>(32 * quarter) << 16;
     const float4* b1 = reinterpret_cast<const float4*>(p.b1[m] + hh * C::HID + g * C::HG);  // group's hidden units
-    const float4* b2 = reinterpret_cast<const float4*>(p.b2[m] + hh * C::OUT + g * C::OG);  // group's features
-    const bool square = g * C::OG >= D;  // features D..2D-1 are psi_2^2
     const int r = 32 * quarter + lane;   // row inside the tile
     const uint32_t my_stg = smem_u32(smem + C::OFF_STG) + g * C::STG_BOX + r * 64;
     const int swz = (r >> 1) & 3;
@@ -167,27 +176,33 @@ __global__ void __launch_bounds__(MlpCfg<D>::THREADS, 1) phi_mlp_kernel(const __
       }
       warp_release(BAR(C::B_R), lane);
       if (threadIdx.x == 0) TRACE(1, it);
-      ok = ok && warp_wait(BAR(C::B_U), it & 1, abort);
-      if (threadIdx.x == 0) TRACE(2, it);
-      tc_fence_after();
       // phi = psi(U + b2), squared for the second half, one row a thread,
       // staged in shared memory (64-byte swizzle: 16-byte chunk j of row r at
       // chunk j ^ ((r >> 1) & 3)); the producer thread stores each step by TMA
 #pragma unroll 1
       for (int c = 0; c < C::NC; ++c) {
+        const int uh = C::SPLIT ? c : 0;  // U half of this chunk
+        const int fc = C::SPLIT ? c * (C::OUT / 2) + 32 * g : g * C::OG + 32 * c;  // its first feature
+        if (C::SPLIT || c == 0) {
+          ok = ok && warp_wait(BAR(C::B_U + uh), it & 1, abort);
+          if (c == 0 && threadIdx.x == 0) TRACE(2, it);
+          tc_fence_after();
+        }
         uint32_t v[32];
-        tmem_ld32(tmem + lane_off + C::HID + g * C::OG + 32 * c, v);
+        tmem_ld32(tmem + lane_off + C::HID + fc, v);
         tmem_ld_wait();
         reg_fence(v);
-        if (c == C::NC - 1) {  // U fully read: the next tile's second GEMM may overwrite it
+        if (C::SPLIT || c == C::NC - 1) {  // U (half) fully read: the next tile's GEMM may overwrite it
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(BAR(C::B_UE));
+          if (lane == 0) mbar_arrive(BAR(C::B_UE + uh));
         }
+        const float4* b2 = reinterpret_cast<const float4*>(p.b2[m] + hh * C::OUT + fc);
+        const bool square = fc >= D;  // features D..2D-1 are psi_2^2
         uint32_t o[16];
 #pragma unroll
         for (int q4 = 0; q4 < 8; ++q4) {
-          const float4 bv = __ldg(b2 + 8 * c + q4);
+          const float4 bv = __ldg(b2 + q4);
           const float u0 = __uint_as_float(v[4 * q4]) + bv.x, u1 = __uint_as_float(v[4 * q4 + 1]) + bv.y;
           const float u2 = __uint_as_float(v[4 * q4 + 2]) + bv.z, u3 = __uint_as_float(v[4 * q4 + 3]) + bv.w;
           float f0 = psi1(u0), f1 = psi1(u1), f2 = psi1(u2), f3 = psi1(u3);
@@ -249,8 +264,9 @@ __global__ void __launch_bounds__(MlpCfg<D>::THREADS, 1) phi_mlp_kernel(const __
           if (!ok) break;
           const uint32_t stg0 = smem_u32(smem + C::OFF_STG);
           for (int gg = 0; gg < C::NG; ++gg)
-            tma_store_3d(&p.tm_phi[m], stg0 + gg * C::STG_BOX, gg * C::OG + 32 * c, 128 * (grp_id + it * p.groups),
-                         bh);
+            tma_store_3d(&p.tm_phi[m], stg0 + gg * C::STG_BOX,
+                         C::SPLIT ? c * (C::OUT / 2) + 32 * gg : gg * C::OG + 32 * c,
+                         128 * (grp_id + it * p.groups), bh);
           bulk_commit();
           TRACE(5 + (c & 1), it);
           bulk_wait_read<0>();  // the staging area may be written again
@@ -277,7 +293,7 @@ __global__ void __launch_bounds__(MlpCfg<D>::THREADS, 1) phi_mlp_kernel(const __
         // H overwrites the TMEM columns that hold R of the previous tile, the
         // A operand of its second GEMM: issued only once that GEMM has
         // completed (tcgen05 operands must not change under an MMA in flight)
-        if (ok && it > 0) ok = mbar_wait(BAR(C::B_U), (it - 1) & 1, abort);
+        if (ok && it > 0) ok = mbar_wait(BAR(C::B_U + C::NU - 1), (it - 1) & 1, abort);
         if (!ok) break;
         TRACE(8, it);
         tc_fence_after();
@@ -289,18 +305,24 @@ __global__ void __launch_bounds__(MlpCfg<D>::THREADS, 1) phi_mlp_kernel(const __
         mma_commit(BAR(C::B_XE + slot));
         mma_commit(BAR(C::B_H));
         TRACE(9, it);
-        // R of this tile written, and U free (the previous tile's features stored)
-        ok = mbar_wait(BAR(C::B_R), it & 1, abort) && mbar_wait(BAR(C::B_UE), (it & 1) ^ 1, abort);
-        if (!ok) break;
-        TRACE(10, it);
-        tc_fence_after();
+        // R of this tile written; each U half once the previous tile's
+        // features of that half have been read out of it
+        ok = mbar_wait(BAR(C::B_R), it & 1, abort);
+        for (int h = 0; h < C::NU && ok; ++h) {
+          ok = mbar_wait(BAR(C::B_UE + h), (it & 1) ^ 1, abort);
+          if (!ok) break;
+          if (h == 0) TRACE(10, it);
+          tc_fence_after();
+          const uint32_t wrow = (h * (C::OUT / C::NU) * 128) >> 4;  // the half's first W2 row
 #pragma unroll
-        for (int kk = 0; kk < C::HID / 16; ++kk) {  // 16 hidden units = 8 packed columns of R
-          const uint32_t a = tmem + (kk / (C::HG / 16)) * C::HG + (kk % (C::HG / 16)) * 8;
-          mma_ts(tmem + C::HID, a, desc_join(lo_w2 + (((kk >> 2) * C::W2BOX + (kk & 3) * 32) >> 4), HI), C::IDESC2,
-                 kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < C::HID / 16; ++kk) {  // 16 hidden units = 8 packed columns of R
+            const uint32_t a = tmem + (kk / (C::HG / 16)) * C::HG + (kk % (C::HG / 16)) * 8;
+            mma_ts(tmem + C::HID + h * (C::OUT / C::NU), a,
+                   desc_join(lo_w2 + wrow + (((kk >> 2) * C::W2BOX + (kk & 3) * 32) >> 4), HI), C::IDESC2,
+                   kk > 0 ? 1u : 0u);
+          }
+          mma_commit(BAR(C::B_U + h));
         }
-        mma_commit(BAR(C::B_U));
       }
       mma_commit(BAR(C::B_FIN));
       drain_wait(BAR(C::B_FIN), 0);
