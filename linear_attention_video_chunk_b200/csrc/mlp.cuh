@@ -19,7 +19,6 @@ struct MlpParams {
   const float* b1[2];     // [H, 2D]
   const float* b2[2];     // [H, 2D]
   __nv_bfloat16* phi[2];  // [BH, N, 2D]
-  CUtensorMap tm_phi[2];  // phi as 3-D {2D, N, BH}, box {32, 128, 1}, 64-byte swizzle (stores)
   int N, H, BH, groups;
   unsigned long long* trace;  // clock64 stamps, only with -DREHYAT_TRACE (else unused)
 };

@@ -27,13 +27,12 @@ namespace {
 // column group w / 4 (a quarter of H's and of U's columns); warp 16 is the TMA
 // producer, warp 17 the MMA issuer.  The next H GEMM (issued once the second
 // GEMM, which reads R from H's columns, has completed) runs while the
-// epilogue still reads U.  Features leave through shared memory and TMA tile stores
-// (32 features x 128 rows a box, one box per group and chunk step), so each
-// row is written whole instead of 16 bytes per thread at a 2D-element
-// stride; the producer thread issues those stores and waits for them, so the
-// epilogue warps never block on a store.  At D = 128 the weights leave room
-// for one x tile only, and the staging area is that tile once the next H GEMM
-// has read it.
+// epilogue still reads U.  Features leave straight from registers: a thread
+// holds 32 features (four 16-byte parts) of its row, the four threads of a
+// lane quad exchange parts (a 4 x 4 transpose in two xor shuffles), and each
+// store instruction then writes 64 contiguous bytes of each of 8 rows.  With
+// no staging area in shared memory (at D = 128 the weights leave room for one
+// x tile only) the next x tile loads as soon as the H GEMM has read the last.
 template <int D>
 struct MlpCfg {
   static constexpr int HID = 2 * D;                 // hidden width
@@ -50,14 +49,10 @@ struct MlpCfg {
   static constexpr int NG = 4;                      // epilogue column groups
   static constexpr int HG = HID / NG;               // hidden units of a group
   static constexpr int OG = OUT / NG;               // features of a group
-  static constexpr int STG_BOX = 128 * 64;          // 32 features x 128 rows, bf16
-  static constexpr int STG_STEP = NG * STG_BOX;     // one chunk step of every group
-  static constexpr bool ALIAS = (D == 128);         // staging = the (single) x tile buffer
   static constexpr int OFF_W1 = 0;
   static constexpr int OFF_W2 = W1_BYTES;
   static constexpr int OFF_X = OFF_W2 + W2_BYTES;
-  static constexpr int OFF_STG = ALIAS ? OFF_X : OFF_X + NXB * X_BYTES;
-  static constexpr int OFF_BAR = ALIAS ? OFF_X + NXB * X_BYTES : OFF_STG + STG_STEP;
+  static constexpr int OFF_BAR = OFF_X + NXB * X_BYTES;
   static constexpr int SMEM = OFF_BAR + 256 + 1024;
   static constexpr uint32_t TMEM_COLS = (HID + OUT <= 256) ? 256u : 512u;
   static constexpr int EPI_WARPS = 4 * NG;
@@ -71,10 +66,9 @@ struct MlpCfg {
   static constexpr bool SPLIT = (D == 128);
   static constexpr int NU = SPLIT ? 2 : 1;          // U halves
   static constexpr int B_W = 0, B_X = 1, B_XE = 1 + NXB, B_H = 1 + 2 * NXB, B_R = B_H + 1, B_U = B_H + 2,
-                       B_UE = B_U + 2, B_STF = B_UE + 2, B_STE = B_STF + 1, B_FIN = B_STE + 1;
+                       B_UE = B_U + 2, B_FIN = B_UE + 2;
   static constexpr int NC = OG / 32;                // 32-feature chunk steps of a tile
   static_assert(!SPLIT || NC == NU, "one chunk per U half");
-  static_assert(!ALIAS || (NXB == 1 && X_BYTES >= STG_STEP), "staging inside the x tile");
   static_assert(HG % 32 == 0 && OG % 32 == 0, "whole 32-column chunks per group");
   // both GEMMs: A and B K-major (x rows / R rows by W rows)
   static constexpr uint32_t IDESC1 = idesc_bf16_f32(128, HID, 0, 0);
@@ -118,8 +112,6 @@ __global__ void __launch_bounds__(MlpCfg<D>::THREADS, 1) phi_mlp_kernel(const __
       mbar_init(BAR(C::B_U + h), 1);
       mbar_init(BAR(C::B_UE + h), C::EPI_WARPS);
     }
-    mbar_init(BAR(C::B_STF), C::EPI_WARPS);
-    mbar_init(BAR(C::B_STE), 1);
     mbar_init(BAR(C::B_FIN), 1);
     *abort = 0;
     fence_mbar_init();
@@ -128,7 +120,6 @@ __global__ void __launch_bounds__(MlpCfg<D>::THREADS, 1) phi_mlp_kernel(const __
     prefetch_tmap(&p.tm_x[m]);
     prefetch_tmap(&p.tm_w1[m]);
     prefetch_tmap(&p.tm_w2[m]);
-    prefetch_tmap(&p.tm_phi[m]);
   }
   if (warp == C::EPI_WARPS + 1) {
     tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
@@ -144,12 +135,86 @@ __global__ void __launch_bounds__(MlpCfg<D>::THREADS, 1) phi_mlp_kernel(const __
     const int quarter = warp & 3, g = warp >> 2;
     const uint32_t lane_off = static_cast<uint32_t>(32 * quarter) << 16;
     const float4* b1 = reinterpret_cast<const float4*>(p.b1[m] + hh * C::HID + g * C::HG);  // group's hidden units
-    const int r = 32 * quarter + lane;   // row inside the tile
-    const uint32_t my_stg = smem_u32(smem + C::OFF_STG) + g * C::STG_BOX + r * 64;
-    const int swz = (r >> 1) & 3;
+    const int odd = lane & 1, hi2 = (lane >> 1) & 1;  // position inside the lane quad
     // After a failed wait the remaining waits are skipped and the loop runs
     // out without blocking.
     bool ok = true;
+    // phi = psi(U + b2), squared for the second half, one row a thread: the
+    // 32 features of chunk c of tile t (for c = 0 and at D = 64 the group's
+    // whole share; at D = 128 chunk c is read from U half c)
+    auto feature_chunk = [&](int t, int c) {
+      const int uh = C::SPLIT ? c : 0;  // U half of this chunk
+      const int fc = C::SPLIT ? c * (C::OUT / 2) + 32 * g : g * C::OG + 32 * c;  // its first feature
+      if (C::SPLIT || c == 0) {
+        ok = ok && warp_wait(BAR(C::B_U + uh), t & 1, abort);
+        if (c == 0 && threadIdx.x == 0) TRACE(2, t);
+        tc_fence_after();
+      }
+      uint32_t v[32];
+      tmem_ld32(tmem + lane_off + C::HID + fc, v);
+      tmem_ld_wait();
+      reg_fence(v);
+      if (C::SPLIT || c == C::NC - 1) {  // U (half) fully read: the next tile's GEMM may overwrite it
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(BAR(C::B_UE + uh));
+      }
+      const float4* b2 = reinterpret_cast<const float4*>(p.b2[m] + hh * C::OUT + fc);
+      const bool square = fc >= D;  // features D..2D-1 are psi_2^2
+      uint32_t o[16];
+#pragma unroll
+      for (int q4 = 0; q4 < 8; ++q4) {
+        const float4 bv = __ldg(b2 + q4);
+        const float u0 = __uint_as_float(v[4 * q4]) + bv.x, u1 = __uint_as_float(v[4 * q4 + 1]) + bv.y;
+        const float u2 = __uint_as_float(v[4 * q4 + 2]) + bv.z, u3 = __uint_as_float(v[4 * q4 + 3]) + bv.w;
+        float f0 = psi1(u0), f1 = psi1(u1), f2 = psi1(u2), f3 = psi1(u3);
+        if (square) {
+          f0 *= f0;
+          f1 *= f1;
+          f2 *= f2;
+          f3 *= f3;
+        }
+        o[2 * q4] = pack_bf16(f0, f1);
+        o[2 * q4 + 1] = pack_bf16(f2, f3);
+      }
+      if (c == 0 && threadIdx.x == 0) TRACE(3, t);
+      // 4 x 4 transpose of 16-byte parts inside the lane quad: lane 4q + i
+      // then holds part i (features 8i..8i+7) of rows 4q..4q+3 of the warp's
+      // 32, part k of row 4q + k in P[k]
+      uint4 P[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) P[j] = make_uint4(o[4 * j], o[4 * j + 1], o[4 * j + 2], o[4 * j + 3]);
+      {
+        const uint4 r0 = shfl_xor_u4(odd ? P[0] : P[1], 1), r1 = shfl_xor_u4(odd ? P[2] : P[3], 1);
+        if (odd) {
+          P[0] = r0;
+          P[2] = r1;
+        } else {
+          P[1] = r0;
+          P[3] = r1;
+        }
+      }
+      {
+        const uint4 r0 = shfl_xor_u4(hi2 ? P[0] : P[2], 2), r1 = shfl_xor_u4(hi2 ? P[1] : P[3], 2);
+        if (hi2) {
+          P[0] = r0;
+          P[1] = r1;
+        } else {
+          P[2] = r0;
+          P[3] = r1;
+        }
+      }
+      const int row0 = 128 * (grp_id + t * p.groups) + 32 * quarter + 4 * (lane >> 2);
+      __nv_bfloat16* dst = p.phi[m] + (static_cast<size_t>(bh) * p.N + row0) * C::OUT + fc + 8 * (lane & 3);
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        if (row0 + k < p.N) *reinterpret_cast<uint4*>(dst + static_cast<size_t>(k) * C::OUT) = P[k];
+      if (c == 0 && threadIdx.x == 0) TRACE(4, t);
+    };
+    // Per tile: R, then (at D = 128) the previous tile's second chunk, during
+    // which the tensor core computes this tile's first U half, then this
+    // tile's first chunk, during which it computes the second U half and the
+    // next tile's H.
     for (int it = 0; it < my_tiles; ++it) {
       ok = ok && warp_wait(BAR(C::B_H), it & 1, abort);
       if (threadIdx.x == 0) TRACE(0, it);
@@ -176,63 +241,17 @@ __global__ void __launch_bounds__(MlpCfg<D>::THREADS, 1) phi_mlp_kernel(const __
       }
       warp_release(BAR(C::B_R), lane);
       if (threadIdx.x == 0) TRACE(1, it);
-      // phi = psi(U + b2), squared for the second half, one row a thread,
-      // staged in shared memory (64-byte swizzle: 16-byte chunk j of row r at
-      // chunk j ^ ((r >> 1) & 3)); the producer thread stores each step by TMA
+      if (C::SPLIT) {
+        if (it > 0) feature_chunk(it - 1, 1);
+        feature_chunk(it, 0);
+      } else {
 #pragma unroll 1
-      for (int c = 0; c < C::NC; ++c) {
-        const int uh = C::SPLIT ? c : 0;  // U half of this chunk
-        const int fc = C::SPLIT ? c * (C::OUT / 2) + 32 * g : g * C::OG + 32 * c;  // its first feature
-        if (C::SPLIT || c == 0) {
-          ok = ok && warp_wait(BAR(C::B_U + uh), it & 1, abort);
-          if (c == 0 && threadIdx.x == 0) TRACE(2, it);
-          tc_fence_after();
-        }
-        uint32_t v[32];
-        tmem_ld32(tmem + lane_off + C::HID + fc, v);
-        tmem_ld_wait();
-        reg_fence(v);
-        if (C::SPLIT || c == C::NC - 1) {  // U (half) fully read: the next tile's GEMM may overwrite it
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(BAR(C::B_UE + uh));
-        }
-        const float4* b2 = reinterpret_cast<const float4*>(p.b2[m] + hh * C::OUT + fc);
-        const bool square = fc >= D;  // features D..2D-1 are psi_2^2
-        uint32_t o[16];
-#pragma unroll
-        for (int q4 = 0; q4 < 8; ++q4) {
-          const float4 bv = __ldg(b2 + q4);
-          const float u0 = __uint_as_float(v[4 * q4]) + bv.x, u1 = __uint_as_float(v[4 * q4 + 1]) + bv.y;
-          const float u2 = __uint_as_float(v[4 * q4 + 2]) + bv.z, u3 = __uint_as_float(v[4 * q4 + 3]) + bv.w;
-          float f0 = psi1(u0), f1 = psi1(u1), f2 = psi1(u2), f3 = psi1(u3);
-          if (square) {
-            f0 *= f0;
-            f1 *= f1;
-            f2 *= f2;
-            f3 *= f3;
-          }
-          o[2 * q4] = pack_bf16(f0, f1);
-          o[2 * q4 + 1] = pack_bf16(f2, f3);
-        }
-        if (c == 0 && threadIdx.x == 0) TRACE(3, it);
-        if (c == 0 && C::ALIAS && it + 1 < my_tiles)  // staging = x tile: the next H GEMM has read it
-          ok = ok && warp_wait(BAR(C::B_XE), (it + 1) & 1, abort);
-        const int step = it * C::NC + c;  // staging use; the previous one must have been stored
-        ok = ok && warp_wait(BAR(C::B_STE), (step & 1) ^ 1, abort);
-        if (c == 0 && threadIdx.x == 0) TRACE(4, it);
-#pragma unroll
-        for (int j = 0; j < 4; ++j)
-          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(my_stg + ((j ^ swz) << 4)), "r"(o[4 * j]),
-                       "r"(o[4 * j + 1]), "r"(o[4 * j + 2]), "r"(o[4 * j + 3])
-                       : "memory");
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(BAR(C::B_STF));
+        for (int c = 0; c < C::NC; ++c) feature_chunk(it, c);
       }
     }
+    if (C::SPLIT) feature_chunk(my_tiles - 1, 1);
   } else if (warp == C::EPI_WARPS) {
-    // ================ TMA producer: x tiles in, features out ================
+    // ========================= TMA producer: x tiles =========================
     if (lane == 0) {
       mbar_arrive_expect_tx(BAR(C::B_W), C::W1_BYTES + C::W2_BYTES);
       for (int b = 0; b < C::NBX; ++b)
@@ -242,12 +261,11 @@ __global__ void __launch_bounds__(MlpCfg<D>::THREADS, 1) phi_mlp_kernel(const __
       bool ok = true;
       int loaded = 0;  // x tiles issued
       // x tile `it` into its slot once the H GEMM of the slot's previous tile
-      // has read it (aliased: and once the features staged there have been
-      // stored, which program order below guarantees)
-      auto load_x = [&](int it) {
+      // has read it
+      for (int it = 0; it < my_tiles && ok; ++it) {
         const int slot = it % C::NXB;
-        ok = ok && mbar_wait(BAR(C::B_XE + slot), ((it / C::NXB) & 1) ^ 1, abort);
-        if (!ok) return;
+        ok = mbar_wait(BAR(C::B_XE + slot), ((it / C::NXB) & 1) ^ 1, abort);
+        if (!ok) break;
         TRACE(11, it);
         const uint32_t dst = smem_u32(smem + C::OFF_X + slot * C::X_BYTES);
         mbar_arrive_expect_tx(BAR(C::B_X + slot), C::X_BYTES);
@@ -255,27 +273,7 @@ __global__ void __launch_bounds__(MlpCfg<D>::THREADS, 1) phi_mlp_kernel(const __
           tma_load_4d(dst + b * C::XBOX, &p.tm_x[m], BAR(C::B_X + slot), 64 * b, 128 * (grp_id + it * p.groups), hh,
                       bb);
         loaded = it + 1;
-      };
-      for (int it = 0; it < my_tiles && it < 2; ++it) load_x(it);
-      for (int it = 0; it < my_tiles && ok; ++it) {
-        for (int c = 0; c < C::NC && ok; ++c) {
-          const int step = it * C::NC + c;
-          ok = mbar_wait(BAR(C::B_STF), step & 1, abort);
-          if (!ok) break;
-          const uint32_t stg0 = smem_u32(smem + C::OFF_STG);
-          for (int gg = 0; gg < C::NG; ++gg)
-            tma_store_3d(&p.tm_phi[m], stg0 + gg * C::STG_BOX,
-                         C::SPLIT ? c * (C::OUT / 2) + 32 * gg : gg * C::OG + 32 * c,
-                         128 * (grp_id + it * p.groups), bh);
-          bulk_commit();
-          TRACE(5 + (c & 1), it);
-          bulk_wait_read<0>();  // the staging area may be written again
-          mbar_arrive(BAR(C::B_STE));
-        }
-        TRACE(7, it);
-        if (it + 2 < my_tiles) load_x(it + 2);
       }
-      bulk_wait<0>();  // every feature row written before the CTA exits
       drain_wait(BAR(C::B_W), 0);
       for (int i2 = (loaded > C::NXB ? loaded - C::NXB : 0); i2 < loaded; ++i2)
         drain_wait(BAR(C::B_X + i2 % C::NXB), (i2 / C::NXB) & 1);

@@ -274,21 +274,6 @@ bool make_map4(CUtensorMap* m, const void* base, long long inner, long long rows
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// bf16 [depth, rows, inner] written by TMA tile stores: boxes of 32 x 128,
-// 64-byte swizzle (the staging layout of the feature-map kernel).
-bool make_store_map(CUtensorMap* m, void* base, long long inner, long long rows, long long depth) {
-  EncodeTiledFn fn = encode_fn();
-  if (fn == nullptr) return false;
-  cuuint64_t dims[3] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(rows),
-                        static_cast<cuuint64_t>(depth)};
-  cuuint64_t strides[2] = {static_cast<cuuint64_t>(inner) * 2, static_cast<cuuint64_t>(inner) * 2 * rows};
-  cuuint32_t box[3] = {32u, 128u, 1u};
-  cuuint32_t estr[3] = {1u, 1u, 1u};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-            CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 int cuda_status(cudaError_t e) { return e == cudaSuccess ? REHYAT_OK : REHYAT_ECUDA; }
 
 #ifdef REHYAT_TRACE
@@ -404,8 +389,7 @@ int run_phi_mlp(const MlpArgs* maps, int n_maps, int B, int H, int N, int d, lon
   for (int i = 0; i < n_maps; ++i) {
     if (!make_map4(&mp.tm_x[i], maps[i].x, d, N, H, B, rs, hs, bs, 128) ||
         !make_map(&mp.tm_w1[i], maps[i].W1, d, D2, H, static_cast<int>(D2)) ||
-        !make_map(&mp.tm_w2[i], maps[i].W2, D2, D2, H, static_cast<int>(D2)) ||
-        !make_store_map(&mp.tm_phi[i], maps[i].phi, D2, N, static_cast<long long>(B) * H))
+        !make_map(&mp.tm_w2[i], maps[i].W2, D2, D2, H, static_cast<int>(D2)))
       return REHYAT_ECUDA;
     mp.b1[i] = maps[i].b1;
     mp.b2[i] = maps[i].b2;
