@@ -68,6 +68,11 @@ MLP_CASES = [
     (2, 2, 257, 64, "bhnd", "random", 3),           # d = 64, one-row last tile
     (1, 1, 128, 64, "bnhd", "near_identity", 4),    # exactly one tile
     (1, 1, 5, 128, "bhnd", "random", 5),            # fewer rows than a tile
+    # 80 (map, b.h) pairs: one row group each, so every CTA walks all the
+    # tiles of its head (the cross-tile overlap of the second U half and the
+    # x reloads), the last one ragged
+    (2, 40, 1000, 128, "bhnd", "random", 6),        # 8 tiles, 104-row last tile
+    (1, 80, 700, 64, "bnhd", "near_identity", 7),   # d = 64: 6 tiles, 60-row last tile
 ]
 
 
