@@ -152,19 +152,17 @@ cudaError_t launch_state_scan(const float* part_S, const float* part_z, int BH, 
 cudaError_t launch_state_scan_bidir(const float* part_S, const float* part_z, int BH, int F, int nsplit,
                                     int n_chunks, int D, int Tc, int To, __nv_bfloat16* hi, __nv_bfloat16* lo,
                                     float* Sf, float* zt, cudaStream_t s);
-// state_S/z += sum over pieces of one segment's partials.
 // Combine the two key-window halves of every split unit (AttnParams): out =
 // (O0 2^(m0-M) + O1 2^(m1-M)) / (L0 2^(m0-M) + L1 2^(m1-M)), M = max(m0, m1).
 cudaError_t launch_split_merge(const float* part, int n_split, int split_begin, int BH, int H, int N_q, int D,
                                __nv_bfloat16* out, long long o_sb, long long o_sh, long long o_sr, cudaStream_t s,
                                bool pdl);
+// state_S/z += sum over pieces of one segment's partials.
 cudaError_t launch_state_accumulate(const float* part_S, const float* part_z, int BH, int nsplit,
                                     int D, float* state_S, float* state_z, cudaStream_t s, bool pdl = false);
 // fp32 state -> bf16 hi/lo pair.
 cudaError_t launch_state_split(const float* S, long long n, __nv_bfloat16* hi, __nv_bfloat16* lo,
                                cudaStream_t s);
-
-// The FMA-pipe exp2 used for part of the softmax exponentials (diagnostic).
 
 cudaError_t launch_attention_f32(const AttnF32Params& p, int n_chunks, cudaStream_t s);
 cudaError_t launch_chunk_state_f32(const StateF32Params& p, cudaStream_t s);
