@@ -14,6 +14,19 @@
 namespace rehyat {
 namespace {
 
+// 1 + elu of two values, the multiplies and adds done as packed fp32x2
+// FMAs (x * log2e + 0 and x * 1 + 1 round exactly as the scalar multiply and
+// add), squared as well for the psi^2 features.
+__device__ __forceinline__ void psi_pair(float x0, float x1, bool square, float& f0, float& f1) {
+  const uint64_t l2e2 = pack_f32x2(kLog2e, kLog2e), one2 = pack_f32x2(1.f, 1.f), zero2 = pack_f32x2(0.f, 0.f);
+  float t0, t1, a0, a1;
+  fma_f32x2(__float_as_uint(x0), __float_as_uint(x1), l2e2, zero2, t0, t1);
+  fma_f32x2(__float_as_uint(x0), __float_as_uint(x1), one2, one2, a0, a1);
+  f0 = x0 > 0.f ? a0 : ex2(t0);
+  f1 = x1 > 0.f ? a1 : ex2(t1);
+  if (square) fma_f32x2(__float_as_uint(f0), __float_as_uint(f1), pack_f32x2(f0, f1), zero2, f0, f1);
+}
+
 // ============================================================================
 // Learned feature map: phi = [psi(u_1), psi(u_2)^2], u = W2 relu(W1 x + b1) + b2
 // ============================================================================
@@ -165,15 +178,13 @@ __global__ void __launch_bounds__(MlpCfg<D>::THREADS, 1) phi_mlp_kernel(const __
 #pragma unroll
       for (int q4 = 0; q4 < 8; ++q4) {
         const float4 bv = __ldg(b2 + q4);
-        const float u0 = __uint_as_float(v[4 * q4]) + bv.x, u1 = __uint_as_float(v[4 * q4 + 1]) + bv.y;
-        const float u2 = __uint_as_float(v[4 * q4 + 2]) + bv.z, u3 = __uint_as_float(v[4 * q4 + 3]) + bv.w;
-        float f0 = psi1(u0), f1 = psi1(u1), f2 = psi1(u2), f3 = psi1(u3);
-        if (square) {
-          f0 *= f0;
-          f1 *= f1;
-          f2 *= f2;
-          f3 *= f3;
-        }
+        const uint64_t one2 = pack_f32x2(1.f, 1.f);
+        float u0, u1, u2, u3;  // U + b2
+        fma_f32x2(v[4 * q4], v[4 * q4 + 1], one2, pack_f32x2(bv.x, bv.y), u0, u1);
+        fma_f32x2(v[4 * q4 + 2], v[4 * q4 + 3], one2, pack_f32x2(bv.z, bv.w), u2, u3);
+        float f0, f1, f2, f3;
+        psi_pair(u0, u1, square, f0, f1);
+        psi_pair(u2, u3, square, f2, f3);
         o[2 * q4] = pack_bf16(f0, f1);
         o[2 * q4 + 1] = pack_bf16(f2, f3);
       }
@@ -232,10 +243,12 @@ __global__ void __launch_bounds__(MlpCfg<D>::THREADS, 1) phi_mlp_kernel(const __
 #pragma unroll
         for (int q4 = 0; q4 < 8; ++q4) {
           const float4 bv = __ldg(b1 + 8 * c + q4);
-          rr[2 * q4] = pack_bf16(fmaxf(__uint_as_float(v[4 * q4]) + bv.x, 0.f),
-                                 fmaxf(__uint_as_float(v[4 * q4 + 1]) + bv.y, 0.f));
-          rr[2 * q4 + 1] = pack_bf16(fmaxf(__uint_as_float(v[4 * q4 + 2]) + bv.z, 0.f),
-                                     fmaxf(__uint_as_float(v[4 * q4 + 3]) + bv.w, 0.f));
+          const uint64_t one2 = pack_f32x2(1.f, 1.f);
+          float h0, h1, h2, h3;  // H + b1 (x * 1 + b rounds as x + b)
+          fma_f32x2(v[4 * q4], v[4 * q4 + 1], one2, pack_f32x2(bv.x, bv.y), h0, h1);
+          fma_f32x2(v[4 * q4 + 2], v[4 * q4 + 3], one2, pack_f32x2(bv.z, bv.w), h2, h3);
+          rr[2 * q4] = pack_bf16(fmaxf(h0, 0.f), fmaxf(h1, 0.f));
+          rr[2 * q4 + 1] = pack_bf16(fmaxf(h2, 0.f), fmaxf(h3, 0.f));
         }
         tmem_st16(tmem + lane_off + g * C::HG + 16 * c, rr);
       }
